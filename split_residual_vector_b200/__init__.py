@@ -1,0 +1,204 @@
+"""B200-native split residual vector quantiser of the Mimi codec (the tokenizer
+bottleneck behind Moshi): encode 512-d latents to 8 codes per 80 ms frame
+(1 semantic VQ + 7-level acoustic RVQ, 2048 codewords each) and decode them back.
+
+This module is argument marshalling over the C ABI in ``include/mimi_rvq.h``
+(``libmimi_rvq.so``, built by ``build.py``): every step of the computation runs
+in the library's sm_100a kernels. PyTorch supplies device memory and streams
+only. There is no fallback: if the library is missing or fails to load, using
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LATENT_DIM, DIM, CODEBOOK_SIZE, NUM_CODEBOOKS = 512, 256, 2048, 8
+F32, BF16 = 0, 1
+STATUS = {0: "ok", -1: "invalid argument", -2: "out of device memory", -3: "CUDA error",
+          -4: "code out of range", -5: "device is not sm_100", -6: "kernel wait timed out"}
+
+LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmimi_rvq.so")
+EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_encode_ex",
+           "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
+           "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror")
+
+_lib = None
+
+
+class MimiRVQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, 'unknown')} (status {status})")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """Load libmimi_rvq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIBRARY_PATH):
+        raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
+                          "`python -m split_residual_vector_b200.build`")
+    lib = ctypes.CDLL(LIBRARY_PATH)
+    vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.mimi_rvq_create.argtypes = [vp, vp, vp, ctypes.POINTER(vp)]
+    lib.mimi_rvq_create.restype = ci
+    lib.mimi_rvq_destroy.argtypes = [vp]
+    lib.mimi_rvq_destroy.restype = None
+    lib.mimi_rvq_encode.argtypes = [vp, vp, ci, i64, vp, vp]
+    lib.mimi_rvq_encode.restype = ci
+    for name in ("mimi_rvq_encode_ex", "mimi_rvq_encode_scan"):
+        getattr(lib, name).argtypes = [vp, vp, ci, i64, ci, ci, vp, vp]
+        getattr(lib, name).restype = ci
+    lib.mimi_rvq_project.argtypes = [vp, vp, ci, i64, vp, vp]
+    lib.mimi_rvq_project.restype = ci
+    lib.mimi_rvq_decode_ex.argtypes = [vp, vp, i64, ci, vp, vp]
+    lib.mimi_rvq_decode_ex.restype = ci
+    lib.mimi_rvq_encode_step.argtypes = [vp, vp, ci, ci, vp, vp]
+    lib.mimi_rvq_encode_step.restype = ci
+    lib.mimi_rvq_decode.argtypes = [vp, vp, i64, vp, vp]
+    lib.mimi_rvq_decode.restype = ci
+    lib.mimi_rvq_get_error.argtypes = [vp, vp]
+    lib.mimi_rvq_get_error.restype = ci
+    lib.mimi_rvq_stats.argtypes = [vp, vp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    lib.mimi_rvq_stats.restype = ci
+    lib.mimi_rvq_strerror.argtypes = [ci]
+    lib.mimi_rvq_strerror.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return library().mimi_rvq_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MimiRVQError(status, what)
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_flag(t):
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("latents must be float32 or bfloat16")
+
+
+class Quantizer:
+    """A library handle: codebooks [8, 2048, 256], W_in [256, 512], W_out [512, 256]
+    (float32 CUDA tensors, copied at construction)."""
+
+    def __init__(self, codebooks, W_in, W_out):
+        import torch
+        lib = library()
+        cb = codebooks.detach().to(device="cuda", dtype=torch.float32).contiguous()
+        wi = W_in.detach().to(device=cb.device, dtype=torch.float32).contiguous()
+        wo = W_out.detach().to(device=cb.device, dtype=torch.float32).contiguous()
+        assert cb.shape == (NUM_CODEBOOKS, CODEBOOK_SIZE, DIM), cb.shape
+        assert wi.shape == (DIM, LATENT_DIM) and wo.shape == (LATENT_DIM, DIM)
+        self.device = cb.device
+        self._h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(lib.mimi_rvq_create(cb.data_ptr(), wi.data_ptr(), wo.data_ptr(),
+                                       ctypes.byref(self._h)), "mimi_rvq_create")
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            library().mimi_rvq_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _codes_out(self, n, out, n_q=NUM_CODEBOOKS):
+        import torch
+        if out is None:
+            out = torch.empty((n, n_q), dtype=torch.int16, device=self.device)
+        assert out.dtype == torch.int16 and out.is_contiguous() and out.shape == (n, n_q)
+        return out
+
+    @staticmethod
+    def _latents(latents):
+        assert latents.dim() == 2 and latents.shape[1] == LATENT_DIM and latents.is_contiguous()
+        return latents.shape[0], _dtype_flag(latents)
+
+    def encode(self, latents, n_q=NUM_CODEBOOKS, variant=0, out=None, stream=None):
+        """latents [N, 512] float32 / bfloat16 (CUDA) -> codes [N, n_q] int16."""
+        n, dt = self._latents(latents)
+        out = self._codes_out(n, out, n_q)
+        if n_q == NUM_CODEBOOKS and variant == 0:
+            st = library().mimi_rvq_encode(self._h, latents.data_ptr(), dt, n, out.data_ptr(),
+                                           _stream(stream))
+        else:
+            st = library().mimi_rvq_encode_ex(self._h, latents.data_ptr(), dt, n, n_q, variant,
+                                              out.data_ptr(), _stream(stream))
+        _check(st, "mimi_rvq_encode")
+        return out
+
+    def encode_step(self, frames, out=None, stream=None):
+        """frames [B, 512] (one frame per stream) -> codes [B, 8] int16."""
+        b, dt = self._latents(frames)
+        out = self._codes_out(b, out)
+        _check(library().mimi_rvq_encode_step(self._h, frames.data_ptr(), dt, b, out.data_ptr(),
+                                              _stream(stream)), "mimi_rvq_encode_step")
+        return out
+
+    def project(self, latents, out=None, stream=None):
+        """latents [N, 512] -> y = W_in z [N, 256] float32 (the encoder's projection step)."""
+        import torch
+        n, dt = self._latents(latents)
+        if out is None:
+            out = torch.empty((n, DIM), dtype=torch.float32, device=self.device)
+        assert out.dtype == torch.float32 and out.is_contiguous() and out.shape == (n, DIM)
+        _check(library().mimi_rvq_project(self._h, latents.data_ptr(), dt, n, out.data_ptr(),
+                                          _stream(stream)), "mimi_rvq_project")
+        return out
+
+    def encode_scan(self, latents, n_q=NUM_CODEBOOKS, variant=0, out=None, stream=None):
+        """Float32 full-scan encoder on CUDA cores (slow; for comparison)."""
+        n, dt = self._latents(latents)
+        out = self._codes_out(n, out, n_q)
+        _check(library().mimi_rvq_encode_scan(self._h, latents.data_ptr(), dt, n, n_q, variant,
+                                              out.data_ptr(), _stream(stream)),
+               "mimi_rvq_encode_scan")
+        return out
+
+    def decode(self, codes, out=None, stream=None):
+        """codes [N, n_q] int16 (CUDA) -> latents [N, 512] float32 (n_q = codes.shape[1])."""
+        import torch
+        assert codes.dtype == torch.int16 and codes.is_contiguous() and codes.dim() == 2
+        n, n_q = codes.shape
+        if out is None:
+            out = torch.empty((n, LATENT_DIM), dtype=torch.float32, device=self.device)
+        assert out.dtype == torch.float32 and out.is_contiguous() and out.shape == (n, LATENT_DIM)
+        if n_q == NUM_CODEBOOKS:
+            st = library().mimi_rvq_decode(self._h, codes.data_ptr(), n, out.data_ptr(),
+                                           _stream(stream))
+        else:
+            st = library().mimi_rvq_decode_ex(self._h, codes.data_ptr(), n, n_q, out.data_ptr(),
+                                              _stream(stream))
+        _check(st, "mimi_rvq_decode")
+        return out
+
+    def get_error(self, stream=None) -> int:
+        """Synchronise the stream; return and clear the device error status (0 = ok)."""
+        return int(library().mimi_rvq_get_error(self._h, _stream(stream)))
+
+    def stats(self, stream=None):
+        """(frames encoded, frames re-encoded by the float32 full scan) since create."""
+        a, b = ctypes.c_int64(), ctypes.c_int64()
+        _check(library().mimi_rvq_stats(self._h, _stream(stream), ctypes.byref(a),
+                                        ctypes.byref(b)), "mimi_rvq_stats")
+        return a.value, b.value

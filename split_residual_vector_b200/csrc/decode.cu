@@ -1,0 +1,70 @@
+// decode.cu -- codes [N][8] -> latents [N][512] fp32.
+//
+// The decode is x = W_out . (S_s + sum_l A_{l,a_l}). W_out is linear, so
+// x = sum_l P_l[code_l] with P_l = W_out . C_l, a [2048][512] table per
+// codebook built once at create (float64 sums, rounded to float32). The kernel
+// is then a pure gather-sum: one warp per frame, each lane owns 16 of the 512
+// outputs (4 float4 at a 512-byte warp stride, so every load and store is a
+// fully coalesced 512-byte warp transaction). The tables (32 MiB) stay in L2
+// and hot rows in L1; the output is written with evict-first stores so that
+// the 2 KiB/frame output stream does not push the tables out of L2.
+#include "handle.cuh"
+#include "ptx.cuh"
+
+namespace mimi {
+namespace {
+
+constexpr int kWarps = 8;
+
+__global__ void __launch_bounds__(kWarps * 32) k_decode(const float* __restrict__ P,
+                                                        const int16_t* __restrict__ codes,
+                                                        int64_t n, int n_q, float* __restrict__ out,
+                                                        int* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t nwarps = (int64_t)gridDim.x * kWarps;
+    for (int64_t f = warp0; f < n; f += nwarps) {
+        int code = lane < n_q ? (int)codes[f * n_q + lane] : 0;
+        if (lane < n_q && (code < 0 || code >= kK)) {
+            atomicOr(err, MIMI_DEV_ERR_RANGE);
+            code = code < 0 ? 0 : kK - 1;
+        }
+        float4 acc[4];
+#pragma unroll
+        for (int l = 0; l < kQ; ++l) {
+            if (l >= n_q) break;  // quantizer dropout: only the first n_q codebooks
+            const int c = __shfl_sync(0xffffffffu, code, l);
+            const float4* row =
+                reinterpret_cast<const float4*>(P + ((size_t)l * kK + (size_t)c) * kDin);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 v = __ldg(row + lane + 32 * u);
+                if (l == 0) {
+                    acc[u] = v;
+                } else {
+                    acc[u].x += v.x;
+                    acc[u].y += v.y;
+                    acc[u].z += v.z;
+                    acc[u].w += v.w;
+                }
+            }
+        }
+        float4* o = reinterpret_cast<float4*>(out + (size_t)f * kDin);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) __stcs(o + lane + 32 * u, acc[u]);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int n_q, float* out,
+                          cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    int64_t blocks = (n + kWarps - 1) / kWarps;
+    const int64_t cap = 148 * 8;  // 8 resident blocks of 8 warps per SM
+    if (blocks > cap) blocks = cap;
+    k_decode<<<(int)blocks, kWarps * 32, 0, s>>>(t.P, codes, n, n_q, out, t.err);
+    return cudaGetLastError();
+}
+
+}  // namespace mimi

@@ -1,0 +1,543 @@
+// encode_tc.cu -- fused projection + split-RVQ encode on tcgen05 tensor cores.
+//
+// Per tile of 128 frames (one persistent CTA per SM, tiles strided over CTAs):
+//
+//   1. projection y = W_in . z on the tensor cores, in split precision so that
+//      y is float32-accurate: z = z_hi + z_lo and W_in = W_hi + W_lo (bf16
+//      halves; bf16 latents are exact, so z_lo = 0) and
+//      y = z_hi W_hi^T + z_lo W_hi^T + z_hi W_lo^T, accumulated in TMEM
+//      columns [0, 256). Those columns then hold the residual r (float32) for
+//      the whole level chain: it never leaves the SM.
+//   2. for each codebook l = 0 (semantic, on y) and 1..7 (acoustic, on r):
+//      candidate scores ||c||^2 - 2 bf16(r) . bf16(c) for all 2048 codewords
+//      as 16 tcgen05 GEMM tiles [128 x 256] x [256 x 128] (codebook tiles
+//      streamed by TMA into a shared-memory ring; accumulators double-buffered
+//      in TMEM columns [256, 512)). The epilogue keeps a sorted top-8 per row.
+//   3. certified pick: with E a rigorous bound on |bf16 score - exact score|
+//      (from ||r||, max ||c|| of the codebook and the bf16 / fp32 rounding
+//      units), every codeword outside the top-8 is ruled out when
+//      s_8 > s_1 + 2E; the candidates within s_1 + 2E are re-scored in float32
+//      (||c||^2 - 2 r.c with r read from TMEM and c from the float32
+//      codebook); a single candidate needs no re-score. If the top-8 cannot be
+//      certified the frame is queued for the float32 full scan.
+//   4. acoustic levels: r -= c_win in TMEM, and bf16(r) is written into the
+//      shared-memory A operand of the next level.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
+// issues the MMAs (one thread), warps 2..5 are the epilogue (thread = frame row
+// = TMEM lane). The semantic level (0) and acoustic level 1 share the A
+// operand bf16(y), so the tensor core runs from level 0 into level 1 while the
+// epilogue re-scores level 0.
+#include <cuda.h>
+
+#include "handle.cuh"
+#include "ptx.cuh"
+
+namespace mimi {
+namespace {
+
+constexpr int BM = 128;                 // frames per tile = TMEM lanes
+constexpr int BN = 128;                 // codewords per score tile
+constexpr int BK = 64;                  // K elements per stage (128 B of bf16)
+constexpr int NT = kK / BN;             // 16 score tiles per codebook
+constexpr int KCH = kD / BK;            // 4 K chunks per score tile
+constexpr int PKCH = kDin / BK;         // 8 K chunks of the projection
+constexpr int STAGES = 8;
+constexpr int STAGE_BYTES = BN * BK * 2;        // 16 KiB
+constexpr int A_CHUNK_BYTES = BM * BK * 2;      // 16 KiB
+constexpr int RING_OFF = 0;
+constexpr int A_OFF = STAGES * STAGE_BYTES;     // 128 KiB
+constexpr int BAR_OFF = A_OFF + KCH * A_CHUNK_BYTES;  // 192 KiB
+constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;     // barriers, slack for 1 KiB alignment
+constexpr int TOPK = 8;
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
+
+// bound coefficients (see header comment): bf16 rounding of both operands
+// (2 u + u^2, u = 2^-9), fp32 accumulation of 256 products (<= 2^-15 of the
+// absolute sum), times 2 for the -2 r.c, plus slack.
+constexpr float kBoundDot = 0.0080f;
+constexpr float kBoundNorm = 4.8e-7f;   // > 2^-21: fp32 rounding of ||c||^2 and of the score
+
+struct Bars {
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t zfull[2], zempty[2];
+    uint64_t yfull, afull, aempty, drain;
+    uint64_t tfull[2], tempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void insert_top8(float (&ts)[TOPK], int (&ti)[TOPK], float s, int k) {
+#pragma unroll
+    for (int p = 0; p < TOPK; ++p) {
+        if (s < ts[p]) {
+            const float ft = ts[p];
+            const int it = ti[p];
+            ts[p] = s;
+            ti[p] = k;
+            s = ft;
+            k = it;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_encode_tc(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_Whi,
+                const __grid_constant__ CUtensorMap tm_Wlo, const float* __restrict__ C32,
+                const float* __restrict__ cnorm, const float* __restrict__ cbound,
+                const void* __restrict__ z, int dtype, int64_t n, int n_q, int variant,
+                int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
+                int* rescan_count, int* rescan_list, unsigned long long* stats) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
+    volatile int* abort = &bars->abort;
+    const uint32_t ring = smem_u32(smem + RING_OFF);
+    const uint32_t abase = smem_u32(smem + A_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n_tiles = (n + BM - 1) / BM;
+    const bool f32_in = (dtype == 0);
+    // Level l rewrites the A operand (r -= c_win, then bf16(r)) for level l + 1
+    // when the next level quantises a different vector: always for acoustic
+    // levels, and after the semantic level too when the acoustic RVQ runs on
+    // y - S_s (variant 1).
+    auto updates_after = [&](int l) { return l < n_q - 1 && (l >= 1 || variant == 1); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->zfull[b], 4);
+            mbar_init(&bars->zempty[b], 1);
+            mbar_init(&bars->tfull[b], 1);
+            mbar_init(&bars->tempty[b], 4);
+        }
+        mbar_init(&bars->yfull, 1);
+        mbar_init(&bars->afull, 4);
+        mbar_init(&bars->aempty, 1);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_C);
+        prefetch_tmap(&tm_Whi);
+        prefetch_tmap(&tm_Wlo);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            auto load = [&](const CUtensorMap* tm, int x, int y) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(&bars->empty[s], ph ^ 1, abort, err)) return false;
+                mbar_arrive_expect_tx(&bars->full[s], STAGE_BYTES);
+                tma_load_2d(smem + RING_OFF + s * STAGE_BYTES, tm, &bars->full[s], x, y);
+                ++it;
+                return true;
+            };
+            for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                for (int kc = 0; kc < PKCH && ok; ++kc) {
+                    ok = ok && load(&tm_Whi, kc * BK, 0) && load(&tm_Whi, kc * BK, BN);
+                    ok = ok && load(&tm_Wlo, kc * BK, 0) && load(&tm_Wlo, kc * BK, BN);
+                }
+                for (int l = 0; l < n_q && ok; ++l)
+                    for (int nt = 0; nt < NT && ok; ++nt)
+                        for (int kc = 0; kc < KCH && ok; ++kc)
+                            ok = load(&tm_C, kc * BK, l * kK + nt * BN);
+            }
+            // drain: every issued copy must land before the CTA exits
+            const uint32_t first = it > STAGES ? it - STAGES : 0;
+            for (uint32_t j = first; j < it; ++j)
+                mbar_wait(&bars->full[j % STAGES], (j / STAGES) & 1, abort, err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+            uint32_t it = 0, zuse[2] = {0, 0}, acnt = 0, tcnt = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                // projection: y = z_hi W_hi + z_lo W_hi + z_hi W_lo into columns [0, 256)
+                for (int kc = 0; kc < PKCH && ok; ++kc) {
+                    const int zb = kc & 1;
+                    ok = mbar_wait(&bars->zfull[zb], zuse[zb] & 1, abort, err);
+                    ++zuse[zb];
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_hi = abase + zb * 2 * A_CHUNK_BYTES;
+                    const uint32_t a_lo = a_hi + A_CHUNK_BYTES;
+                    for (int g = 0; g < 4 && ok; ++g) {
+                        const int s = it % STAGES;
+                        ok = mbar_wait(&bars->full[s], (it / STAGES) & 1, abort, err);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t b = ring + s * STAGE_BYTES;
+                        const uint32_t d = tmem + (g & 1) * BN;
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            const uint32_t acc = (kc > 0 || k > 0 || g >= 2) ? 1u : 0u;
+                            umma_bf16(d, sw128_desc(a_hi + 32 * k), sw128_desc(b + 32 * k), idesc,
+                                      acc);
+                            if (g < 2 && f32_in)
+                                umma_bf16(d, sw128_desc(a_lo + 32 * k), sw128_desc(b + 32 * k),
+                                          idesc, 1u);
+                        }
+                        umma_commit(&bars->empty[s]);
+                        ++it;
+                    }
+                    umma_commit(&bars->zempty[zb]);
+                }
+                if (!ok) break;
+                umma_commit(&bars->yfull);
+                // the eight codebooks
+                for (int l = 0; l < n_q && ok; ++l) {
+                    if (l == 0 || updates_after(l - 1)) {
+                        ok = mbar_wait(&bars->afull, acnt & 1, abort, err);
+                        ++acnt;
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    for (int nt = 0; nt < NT && ok; ++nt) {
+                        const int bsel = tcnt & 1;
+                        ok = mbar_wait(&bars->tempty[bsel], ((tcnt >> 1) & 1) ^ 1, abort, err);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t d = tmem + TMEM_SCORE + bsel * BN;
+                        for (int kc = 0; kc < KCH && ok; ++kc) {
+                            const int s = it % STAGES;
+                            ok = mbar_wait(&bars->full[s], (it / STAGES) & 1, abort, err);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint32_t b = ring + s * STAGE_BYTES;
+                            const uint32_t a = abase + kc * A_CHUNK_BYTES;
+#pragma unroll
+                            for (int k = 0; k < BK / 16; ++k)
+                                umma_bf16(d, sw128_desc(a + 32 * k), sw128_desc(b + 32 * k), idesc,
+                                          (kc > 0 || k > 0) ? 1u : 0u);
+                            umma_commit(&bars->empty[s]);
+                            ++it;
+                        }
+                        umma_commit(&bars->tfull[bsel]);
+                        ++tcnt;
+                    }
+                    if (updates_after(l) || l == n_q - 1) umma_commit(&bars->aempty);
+                }
+            }
+            // drain: every issued MMA must complete before TMEM is freed
+            umma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0, abort, err);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint32_t zuse[2] = {0, 0}, aecnt = 0, tcnt = 0, tile_iter = 0;
+        bool ok = true;
+        unsigned long long done = 0;
+        // every lane of the warp takes the same branch after a wait, so the
+        // .sync.aligned TMEM loads below are never reached divergently
+        auto ewait = [&](uint64_t* bar, uint32_t parity) {
+            const bool r = mbar_wait(bar, parity, abort, err);
+            return __all_sync(0xffffffffu, r) != 0;
+        };
+        for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tile_iter) {
+            const int64_t frame = tile * BM + row;
+            const bool valid = frame < n;
+            // A region is z staging now: wait until the previous tile's level-7 MMAs are done
+            if (tile_iter > 0 && n_q > 0) {
+                ok = ewait(&bars->aempty, aecnt & 1);
+                ++aecnt;
+                if (!ok) break;
+            }
+            // ---- stage z (split into bf16 hi / lo) for the projection
+            for (int kc = 0; kc < PKCH && ok; ++kc) {
+                const int zb = kc & 1;
+                if (zuse[zb] > 0) {
+                    ok = ewait(&bars->zempty[zb], (zuse[zb] - 1) & 1);
+                    if (!ok) break;
+                }
+                ++zuse[zb];
+                uint8_t* zhi = smem + A_OFF + zb * 2 * A_CHUNK_BYTES;
+                uint8_t* zlo = zhi + A_CHUNK_BYTES;
+                if (f32_in) {
+                    const float4* src =
+                        reinterpret_cast<const float4*>(static_cast<const float*>(z) +
+                                                        (valid ? frame : 0) * kDin + kc * BK);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        float4 u = valid ? __ldg(src + 2 * p) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float4 v = valid ? __ldg(src + 2 * p + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        uint4 h, lo;
+                        h.x = pack_bf16x2(u.x, u.y);
+                        h.y = pack_bf16x2(u.z, u.w);
+                        h.z = pack_bf16x2(v.x, v.y);
+                        h.w = pack_bf16x2(v.z, v.w);
+                        lo.x = pack_bf16x2(u.x - bf16_lo_to_f32(h.x), u.y - bf16_hi_to_f32(h.x));
+                        lo.y = pack_bf16x2(u.z - bf16_lo_to_f32(h.y), u.w - bf16_hi_to_f32(h.y));
+                        lo.z = pack_bf16x2(v.x - bf16_lo_to_f32(h.z), v.y - bf16_hi_to_f32(h.z));
+                        lo.w = pack_bf16x2(v.z - bf16_lo_to_f32(h.w), v.w - bf16_hi_to_f32(h.w));
+                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, p)) = h;
+                        *reinterpret_cast<uint4*>(zlo + sw128_offset(row, p)) = lo;
+                    }
+                } else {
+                    const uint4* src = reinterpret_cast<const uint4*>(
+                        static_cast<const uint16_t*>(z) + (valid ? frame : 0) * kDin + kc * BK);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint4 h = valid ? __ldg(src + p) : make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, p)) = h;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->zfull[zb]);
+            }
+            if (!ok) break;
+            // ---- y from TMEM: norm and the bf16 A operand of levels 0 and 1
+            ok = ewait(&bars->yfull, tile_iter & 1);
+            if (!ok) break;
+            tc_fence_after();
+            float nr2 = 0.f;
+            for (int ch = 0; ch < kD / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld32(trow + ch * 32, v);
+                tmem_wait_ld();
+                if (y_out && valid) {
+                    float4* dst = reinterpret_cast<float4*>(y_out + frame * kD + ch * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                              __uint_as_float(v[4 * q4 + 2]),
+                                              __uint_as_float(v[4 * q4 + 3]));
+                }
+                if (n_q == 0) continue;
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+                    nr2 = fmaf(a, a, nr2);
+                    nr2 = fmaf(b, b, nr2);
+                    pk[i] = pack_bf16x2(a, b);
+                }
+                uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    *reinterpret_cast<uint4*>(dst + sw128_offset(row, (ch & 1) * 4 + p)) =
+                        make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
+            }
+            tc_fence_before();
+            if (n_q == 0) continue;  // projection only: y has been written out
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->afull);
+
+            int win_codes[kQ];
+            bool flagged = false;
+            for (int l = 0; l < n_q && ok; ++l) {
+                float ts[TOPK];
+                int ti[TOPK];
+#pragma unroll
+                for (int p = 0; p < TOPK; ++p) {
+                    ts[p] = __int_as_float(0x7f800000);
+                    ti[p] = 0x7fffffff;
+                }
+                const float* cn = cnorm + (size_t)l * kK;
+                // ---- scan the 16 score tiles of this codebook
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int bsel = tcnt & 1;
+                    ok = ewait(&bars->tfull[bsel], (tcnt >> 1) & 1);
+                    ++tcnt;
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int ch = 0; ch < BN / 32; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(trow + TMEM_SCORE + bsel * BN + ch * 32, v);
+                        tmem_wait_ld();
+                        if (ch == BN / 32 - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
+                        }
+                        const int k0 = nt * BN + ch * 32;
+                        const float4* cn4 = reinterpret_cast<const float4*>(cn + k0);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 c = __ldg(cn4 + q4);
+                            const float s0 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 0]), c.x);
+                            const float s1 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 1]), c.y);
+                            const float s2 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 2]), c.z);
+                            const float s3 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 3]), c.w);
+                            const float m = fminf(fminf(s0, s1), fminf(s2, s3));
+                            if (m < ts[TOPK - 1]) {
+                                insert_top8(ts, ti, s0, k0 + 4 * q4 + 0);
+                                insert_top8(ts, ti, s1, k0 + 4 * q4 + 1);
+                                insert_top8(ts, ti, s2, k0 + 4 * q4 + 2);
+                                insert_top8(ts, ti, s3, k0 + 4 * q4 + 3);
+                            }
+                        }
+                    }
+                }
+                if (!ok) break;
+                // ---- certified window and float32 re-score
+                const float cmax = __ldg(cbound + 2 * l), cnmax = __ldg(cbound + 2 * l + 1);
+                const float nr = sqrtf(nr2) * 1.0001f;
+                const float E = nr * cmax * kBoundDot + cnmax * kBoundNorm;
+                const float thr = ts[0] + 2.f * E;
+                int m = 0;
+#pragma unroll
+                for (int p = 0; p < TOPK; ++p) m += (ts[p] <= thr) ? 1 : 0;
+                if (valid && !(ts[TOPK - 1] > thr) && !flagged) {
+                    flagged = true;
+                    const int slot = atomicAdd(rescan_count, 1);
+                    if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
+                }
+                const float* book = C32 + (size_t)l * kK * kD;
+                int win = ti[0];
+                if (__any_sync(0xffffffffu, m > 1)) {
+                    float dot[TOPK];
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
+                    for (int ch = 0; ch < kD / 32; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(trow + ch * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int p = 0; p < TOPK; ++p) {
+                            if (p < m) {
+                                const float4* c4 = reinterpret_cast<const float4*>(
+                                    book + (size_t)ti[p] * kD + ch * 32);
+                                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                                for (int q4 = 0; q4 < 8; ++q4) {
+                                    const float4 c = __ldg(c4 + q4);
+                                    a0 = fmaf(__uint_as_float(v[4 * q4 + 0]), c.x, a0);
+                                    a1 = fmaf(__uint_as_float(v[4 * q4 + 1]), c.y, a1);
+                                    a0 = fmaf(__uint_as_float(v[4 * q4 + 2]), c.z, a0);
+                                    a1 = fmaf(__uint_as_float(v[4 * q4 + 3]), c.w, a1);
+                                }
+                                dot[p] += a0 + a1;
+                            }
+                        }
+                    }
+                    float best = __int_as_float(0x7f800000);
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) {
+                        if (p < m) {
+                            const float e = fmaf(-2.f, dot[p], __ldg(cn + ti[p]));
+                            if (e < best || (e == best && ti[p] < win)) {
+                                best = e;
+                                win = ti[p];
+                            }
+                        }
+                    }
+                }
+                if (win < 0 || win >= kK) win = 0;  // only reachable with NaN / Inf inputs
+                win_codes[l] = win;
+                // ---- residual update r -= c_win (levels feeding another level)
+                if (updates_after(l)) {
+                    ok = ewait(&bars->aempty, aecnt & 1);
+                    ++aecnt;
+                    if (!ok) break;
+                    nr2 = 0.f;
+                    const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD);
+                    for (int ch = 0; ch < kD / 32; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(trow + ch * 32, v);
+                        float4 c[8];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) c[q4] = __ldg(c4 + ch * 8 + q4);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            v[4 * q4 + 0] = __float_as_uint(__uint_as_float(v[4 * q4 + 0]) - c[q4].x);
+                            v[4 * q4 + 1] = __float_as_uint(__uint_as_float(v[4 * q4 + 1]) - c[q4].y);
+                            v[4 * q4 + 2] = __float_as_uint(__uint_as_float(v[4 * q4 + 2]) - c[q4].z);
+                            v[4 * q4 + 3] = __float_as_uint(__uint_as_float(v[4 * q4 + 3]) - c[q4].w);
+                        }
+                        tmem_st32(trow + ch * 32, v);
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float a = __uint_as_float(v[2 * i]);
+                            const float b = __uint_as_float(v[2 * i + 1]);
+                            nr2 = fmaf(a, a, nr2);
+                            nr2 = fmaf(b, b, nr2);
+                            pk[i] = pack_bf16x2(a, b);
+                        }
+                        uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
+#pragma unroll
+                        for (int p = 0; p < 4; ++p)
+                            *reinterpret_cast<uint4*>(dst + sw128_offset(row, (ch & 1) * 4 + p)) =
+                                make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
+                    }
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->afull);
+                }
+            }
+            if (!ok) break;
+            tc_fence_before();
+            if (valid && n_q != kQ) {
+                for (int l = 0; l < n_q; ++l) codes[frame * n_q + l] = (int16_t)win_codes[l];
+                ++done;
+            } else if (valid) {
+                uint4 pk;
+                pk.x = (uint32_t)(uint16_t)win_codes[0] | ((uint32_t)(uint16_t)win_codes[1] << 16);
+                pk.y = (uint32_t)(uint16_t)win_codes[2] | ((uint32_t)(uint16_t)win_codes[3] << 16);
+                pk.z = (uint32_t)(uint16_t)win_codes[4] | ((uint32_t)(uint16_t)win_codes[5] << 16);
+                pk.w = (uint32_t)(uint16_t)win_codes[6] | ((uint32_t)(uint16_t)win_codes[7] << 16);
+                *reinterpret_cast<uint4*>(codes + frame * kQ) = pk;
+                ++done;
+            }
+        }
+        // count frames (one atomic per warp)
+        for (int o = 16; o > 0; o >>= 1) done += __shfl_xor_sync(0xffffffffu, done, o);
+        if (lane == 0 && done) atomicAdd(&stats[0], done);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace
+
+cudaError_t encode_tc_configure() {
+    return cudaFuncSetAttribute(k_encode_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES);
+}
+
+cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
+                             int variant, int16_t* codes, float* y_out, cudaStream_t s,
+                             int max_ctas) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t tiles = (n + BM - 1) / BM;
+    const int grid = (int)(tiles < max_ctas ? tiles : max_ctas);
+    k_encode_tc<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm,
+                                                   t.cbound, z, dtype, n, n_q, variant, codes,
+                                                   y_out, t.err, t.rescan_count, t.rescan_list,
+                                                   t.stats);
+    return cudaGetLastError();
+}
+
+}  // namespace mimi

@@ -1,0 +1,248 @@
+"""GPU parity of the encode path (tcgen05 kernel + certified re-score + full-scan fallback)
+against the float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import assert_codes_match
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+def quantizer(model):
+    import split_residual_vector_b200 as pkg
+    return pkg.Quantizer(torch.from_numpy(model.C).cuda(), torch.from_numpy(model.W_in).cuda(),
+                         torch.from_numpy(model.W_out).cuda())
+
+
+def to_device(z):
+    if z.dtype == np.uint16:
+        return torch.from_numpy(z.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(z).cuda()
+
+
+@pytest.fixture(scope="module")
+def offline_small():
+    work = synth.offline_batch(n=1000)
+    return work, quantizer(work.model)
+
+
+def test_pr1_reference_with_planted_frames():
+    def accept_factory(model):
+        def accept(row, kind, codes):
+            _, db, ds = oracle.encode(row[None], model.W_in, model.C)
+            lv = sorted(codes)
+            return bool(np.all(ds[0, lv] - db[0, lv] >= 1e-3 * (1.0 + db[0, lv])))
+        return accept
+    work = synth.pr1_reference(accept=accept_factory(synth.pr1_reference().model))
+    q = quantizer(work.model)
+    codes = q.encode(to_device(work.z)).cpu().numpy()
+    assert q.get_error() == 0
+    ref, db, ds = oracle.encode(work.z, work.model.W_in, work.model.C)
+    stats = assert_codes_match(codes, ref, db, ds, "pr1_reference")
+    for f, (kind, planted) in work.planted.items():
+        if kind == "acoustic":
+            assert codes[f, 1:].tolist() == [planted[lvl] for lvl in range(1, 8)]
+        else:
+            assert codes[f, 0] == planted[0]
+    print("pr1_reference", stats)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("n", [1, 127, 128, 129, 300, 777])
+def test_ragged_sizes(offline_small, n, dtype):
+    work, q = offline_small
+    z = work.z[:n] if dtype == "f32" else synth.to_bf16_bits(work.z[:n])
+    codes = q.encode(to_device(z)).cpu().numpy()
+    assert q.get_error() == 0
+    ref, db, ds = oracle.encode(z, work.model.W_in, work.model.C)
+    assert_codes_match(codes, ref, db, ds, f"n={n} {dtype}")
+    assert codes.min() >= 0 and codes.max() < 2048
+
+
+def test_scan_kernel_matches_oracle(offline_small):
+    work, q = offline_small
+    z = work.z[:300]
+    codes = q.encode_scan(to_device(z)).cpu().numpy()
+    ref, db, ds = oracle.encode(z, work.model.W_in, work.model.C)
+    assert_codes_match(codes, ref, db, ds, "scan")
+
+
+def test_tensor_core_and_scan_agree_on_a_large_batch(offline_small):
+    """Both GPU encoders on 20 000 frames: they may only differ on near-ties, which are a few
+    percent of frames at these distributions; check the disagreeing frames with the oracle."""
+    _, q = offline_small
+    work = synth.offline_batch(n=20000, seed=5)
+    q2 = quantizer(work.model)
+    z = to_device(work.z)
+    a = q2.encode(z).cpu().numpy()
+    b = q2.encode_scan(z).cpu().numpy()
+    diff = np.nonzero(np.any(a != b, axis=1))[0]
+    assert len(diff) < 0.05 * len(a)
+    if len(diff):
+        ref, db, ds = oracle.encode(work.z[diff], work.model.W_in, work.model.C)
+        assert oracle.near_tie(db, ds).all(), "tensor-core and scan encoders differ off a near-tie"
+
+
+def test_offline_batch_full_size_sampled():
+    """240 000 fp32 frames encoded in one call (the launch the benchmark times); 1500 sampled
+    frames (including the ragged last tile) checked against the oracle."""
+    work = synth.offline_batch()
+    q = quantizer(work.model)
+    codes = q.encode(to_device(work.z)).cpu().numpy()
+    assert q.get_error() == 0
+    rng = np.random.default_rng(0)
+    idx = np.unique(np.concatenate([rng.choice(len(work.z), 1400, replace=False),
+                                    np.arange(len(work.z) - 100, len(work.z))]))
+    ref, db, ds = oracle.encode(work.z[idx], work.model.W_in, work.model.C)
+    print("offline sampled", assert_codes_match(codes[idx], ref, db, ds, "offline_batch"))
+    enc, rescanned = q.stats()
+    assert enc == len(work.z)
+    assert rescanned <= len(work.z) // 1000
+
+
+def test_bulk_tokenization_bf16_full_size_sampled():
+    work = synth.bulk_tokenization()
+    q = quantizer(work.model)
+    codes = q.encode(to_device(work.z)).cpu().numpy()
+    assert q.get_error() == 0
+    rng = np.random.default_rng(1)
+    idx = np.unique(np.concatenate([rng.choice(len(work.z), 1400, replace=False),
+                                    np.arange(len(work.z) - 64, len(work.z))]))
+    ref, db, ds = oracle.encode(work.z[idx], work.model.W_in, work.model.C)
+    print("bulk sampled", assert_codes_match(codes[idx], ref, db, ds, "bulk_tokenization"))
+
+
+@pytest.mark.parametrize("batch", [1, 16, 128, 1024])
+def test_streaming_step(batch):
+    model, frames = synth.streaming_step(batch, calls=3)
+    q = quantizer(model)
+    for call in range(3):
+        codes = q.encode_step(to_device(np.ascontiguousarray(frames[call]))).cpu().numpy()
+        ref, db, ds = oracle.encode(frames[call], model.W_in, model.C)
+        assert_codes_match(codes, ref, db, ds, f"step B={batch} call {call}")
+    assert q.get_error() == 0
+
+
+# ------------------------------------------------------------------ adversarial inputs
+
+
+def _small_model(seed=31):
+    return synth.make_model(synth.generator(seed))
+
+
+def test_duplicated_codewords_pick_the_lowest_index():
+    model = _small_model()
+    C = model.C
+    C[0, 1500] = C[0, 700]
+    C[3, 2000] = C[3, 9]
+    C[7, 1024] = C[7, 1023]
+    q = quantizer(model)
+    rows = [synth.plant_latent(model, {0: 700}), synth.plant_latent(model, {0: 1500})]
+    rows += [synth.plant_latent(model, {lvl: 9 if lvl == 3 else 5 for lvl in range(1, 8)})]
+    z = np.stack(rows)
+    codes = q.encode(to_device(z)).cpu().numpy()
+    ref, db, ds = oracle.encode(z, model.W_in, C)
+    assert codes[0, 0] == 700 and codes[1, 0] == 700 and ref[0, 0] == 700
+    assert ref[2, 3] == 9 and np.array_equal(codes[2], ref[2])
+    assert np.array_equal(codes[:, 0], ref[:, 0])
+
+
+def test_many_equal_codewords_go_to_the_full_scan():
+    """Twelve identical codewords nearest to the frame: more ties than the top-8 can hold, so
+    the candidate set cannot be certified; the frame must be re-encoded by the full scan and
+    still return the lowest of the tied indices."""
+    model = _small_model(33)
+    tied = [100 + 37 * j for j in range(12)]
+    for j in tied:
+        model.C[0, j] = model.C[0, tied[0]]
+    q = quantizer(model)
+    z = np.stack([synth.plant_latent(model, {0: tied[5]})] * 3)
+    codes = q.encode(to_device(z)).cpu().numpy()
+    assert (codes[:, 0] == tied[0]).all()
+    _, rescanned = q.stats()
+    assert rescanned == 3
+
+
+def test_zero_huge_and_tiny_latents():
+    model = _small_model(35)
+    q = quantizer(model)
+    rng = np.random.default_rng(2)
+    z = np.concatenate([np.zeros((5, 512), np.float32),
+                        (1e4 * rng.standard_normal((5, 512))).astype(np.float32),
+                        (1e-30 * rng.standard_normal((5, 512))).astype(np.float32),
+                        np.full((5, 512), 1e-40, np.float32)])
+    codes = q.encode(to_device(z)).cpu().numpy()
+    assert q.get_error() == 0
+    ref, db, ds = oracle.encode(z, model.W_in, model.C)
+    assert_codes_match(codes, ref, db, ds, "adversarial magnitudes")
+
+
+# ------------------------------------------------------------------ boundary behaviour
+
+
+def test_argument_errors(offline_small):
+    import split_residual_vector_b200 as pkg
+    work, q = offline_small
+    z = to_device(work.z[:4])
+    with pytest.raises(pkg.MimiRVQError) as e:
+        q.encode(torch.from_numpy(work.z[:4]))            # host pointer
+    assert e.value.status == -1
+    flat = torch.empty(4 * 512 + 1, device="cuda")
+    with pytest.raises(pkg.MimiRVQError):
+        q.encode(flat[1:].view(4, 512))                  # 4-byte aligned only
+    empty = q.encode(z[:0])
+    assert empty.shape == (0, 8)
+    lib = pkg.library()
+    assert lib.mimi_rvq_encode(q._h, z.data_ptr(), 7, 4, empty.data_ptr(), None) == -1  # dtype
+    assert lib.mimi_rvq_encode(None, z.data_ptr(), 0, 4, empty.data_ptr(), None) == -1
+    assert q.get_error() == 0
+
+
+# ------------------------------------------------------------------ projection, n_q, variant
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_projection_step_matches_oracle(offline_small, dtype):
+    """y = W_in z from the tensor-core split-precision projection, against float64."""
+    work, q = offline_small
+    z = work.z[:300] if dtype == "f32" else synth.to_bf16_bits(work.z[:300])
+    y = q.project(to_device(z)).cpu().numpy().astype(np.float64)
+    ref = oracle.project(z, work.model.W_in)
+    err = float(np.abs(y - ref).max())
+    print(f"projection {dtype}: max abs error {err:.3e}")
+    assert err <= (1e-4 if dtype == "f32" else 3e-5)
+
+
+@pytest.mark.parametrize("n_q", [1, 2, 5, 8])
+def test_fewer_codebooks(offline_small, n_q):
+    """Quantizer dropout at inference: the first n_q codebooks only."""
+    work, q = offline_small
+    z = work.z[:300]
+    codes = q.encode(to_device(z), n_q=n_q).cpu().numpy()
+    assert codes.shape == (300, n_q)
+    ref, db, ds = oracle.encode(z, work.model.W_in, work.model.C, n_q=n_q)
+    assert_codes_match(codes, ref, db, ds, f"n_q={n_q}")
+    scan = q.encode_scan(to_device(z), n_q=n_q).cpu().numpy()
+    assert_codes_match(scan, ref, db, ds, f"scan n_q={n_q}")
+
+
+def test_semantic_residual_variant():
+    """variant 1: the acoustic RVQ quantises y - S_s; full 8-codeword plants come back whole."""
+    rng = synth.generator(44)
+    model = synth.make_model(rng)
+    q = quantizer(model)
+    z = synth.latents(rng, 200)
+    plants = []
+    for f in range(0, 200, 20):
+        codes_true = {lvl: int(rng.integers(synth.K)) for lvl in range(8)}
+        z[f] = synth.plant_latent(model, codes_true)
+        plants.append((f, [codes_true[lvl] for lvl in range(8)]))
+    codes = q.encode(to_device(z), variant=1).cpu().numpy()
+    ref, db, ds = oracle.encode(z, model.W_in, model.C, variant=1)
+    assert_codes_match(codes, ref, db, ds, "variant 1")
+    for f, true in plants:
+        assert codes[f].tolist() == true
