@@ -1,0 +1,464 @@
+"""Benchmark of the B200 split-RVQ hot path (Mimi tokenizer bottleneck).
+
+A step is one pass of the whole hot path over one batch: encode (projection,
+semantic VQ, 7-level acoustic RVQ, codes) and decode (gather-sum, projection back)
+of the offline-batch workload: 64 streams x 3750 frames = 240 000 fp32 frames.
+Other workloads (--workload) are the 1 048 576-frame bf16 bulk encode, the
+1 048 576-frame decode-heavy decode, and the streaming step.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize(), timed with CUDA events on the stream the kernels run
+on; the max over ranks is reported. Inputs are larger than L2 (they are not
+re-read from L2 between steps). One JSON line is printed by rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FRAME_HZ = 12.5
+ENC_FLOP = 8 * 2 * 2048 * 256 + 2 * 256 * 512     # 8 650 752 per frame
+DEC_FLOP = 2 * 512 * 256                         # 262 144 per frame (+ 1 792 adds)
+DEC_BYTES = 8 * 2 + 512 * 4                      # codes in + fp32 latents out
+METRIC = "RVQ encode/decode frames/s (real-time streams @12.5 Hz) and % of roofline, 1xB200"
+
+WORKLOADS = {
+    "offline_batch": "64 streams x 3750 frames = 240000 fp32 frames; encode to int16 codes "
+                     "[240000,8] then decode to fp32 [240000,512]",
+    "bulk_tokenization": "1048576 bf16 frames [1048576,512]; encode only, int16 codes out",
+    "decode_heavy": "1048576 frames of codes (semantic uniform, acoustic Zipf(1.1)); decode "
+                    "to fp32 [1048576,512]",
+    "streaming": "B concurrent streams, one fp32 frame each per call; encode_step",
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "util": float(parts[4]), "hw": parts[6], "hwt": parts[7],
+                             "swt": parts[8], "pcap": parts[9]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        load = [r for r in rows if r["util"] >= 50] or rows
+        reasons = set()
+        for r in load:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in load), "reasons": sorted(reasons),
+                "samples": len(load)}
+
+
+# --------------------------------------------------------------------- workloads
+
+
+def make_workload(name, rank, frames=None):
+    """Host-side inputs for one rank (weak scaling: every rank gets a full workload).
+    ``frames`` shrinks the workload (profiling captures only; the bench line uses the
+    full size)."""
+    if name == "offline_batch":
+        w = synth.offline_batch(**({"n": frames} if frames else {}), seed=1 + 100 * rank)
+        return {"model": w.model, "z": w.z, "dtype": "f32", "frames": len(w.z)}
+    if name == "bulk_tokenization":
+        w = synth.bulk_tokenization(**({"n": frames} if frames else {}), seed=3 + 100 * rank)
+        return {"model": w.model, "z": w.z, "dtype": "bf16", "frames": len(w.z)}
+    if name == "decode_heavy":
+        model, codes = synth.decode_heavy(**({"n": frames} if frames else {}),
+                                          seed=4 + 100 * rank)
+        return {"model": model, "codes": codes, "frames": len(codes)}
+    raise ValueError(name)
+
+
+def to_device_latents(torch, z, dtype, device):
+    if dtype == "bf16":
+        return torch.from_numpy(z.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(z).to(device)
+
+
+def cpu_baseline(work, name, budget_s=12.0):
+    """The float64 oracle on this host's cores over a bounded sample of the workload."""
+    import oracle
+    m = work["model"]
+    cores = oracle.threads(0)
+
+    def run(n):
+        t0 = time.perf_counter()
+        if name in ("offline_batch", "bulk_tokenization"):
+            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C)
+            if name == "offline_batch":
+                oracle.decode(codes, m.C, m.W_out)
+        else:
+            oracle.decode(work["codes"][:n], m.C, m.W_out)
+        return time.perf_counter() - t0
+
+    n = 64 if name != "decode_heavy" else 4096
+    dt = run(n)
+    n = int(max(n, min(work["frames"], n * budget_s / max(dt, 1e-3))))
+    dt = run(n)
+    what = {"offline_batch": "encode+decode", "bulk_tokenization": "encode",
+            "decode_heavy": "decode"}[name]
+    return {"value": n / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} frames of the workload, {what}, float64 oracle, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import split_residual_vector_b200 as pkg
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    name = args.workload
+    work = make_workload(name, rank, args.frames)
+    m = work["model"]
+    q = pkg.Quantizer(torch.from_numpy(m.C).to(device), torch.from_numpy(m.W_in).to(device),
+                      torch.from_numpy(m.W_out).to(device))
+    n = work["frames"]
+    stream = torch.cuda.current_stream(device)
+    do_enc = name in ("offline_batch", "bulk_tokenization")
+    do_dec = name in ("offline_batch", "decode_heavy")
+    if do_enc:
+        z = to_device_latents(torch, work["z"], work["dtype"], device)
+        codes = torch.empty((n, 8), dtype=torch.int16, device=device)
+    else:
+        codes = torch.from_numpy(work["codes"]).to(device)
+    x = torch.empty((n, 512), dtype=torch.float32, device=device) if do_dec else None
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    enc_ms, dec_ms = [], []
+
+    def step(timed):
+        if do_enc:
+            a, b = ev(), ev()
+            a.record(stream)
+            q.encode(z, out=codes, stream=stream)
+            b.record(stream)
+            if timed:
+                enc_ms.append((a, b))
+        if do_dec:
+            a, b = ev(), ev()
+            a.record(stream)
+            q.decode(codes, out=x, stream=stream)
+            b.record(stream)
+            if timed:
+                dec_ms.append((a, b))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(device)
+    assert q.get_error(stream) == 0
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    start, stop = ev(), ev()
+    with ClockSampler(local_rank) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    elapsed_ms = start.elapsed_time(stop)
+    if dist:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = q.get_error(stream)
+    enc_avg = sum(a.elapsed_time(b) for a, b in enc_ms) / max(len(enc_ms), 1)
+    dec_avg = sum(a.elapsed_time(b) for a, b in dec_ms) / max(len(dec_ms), 1)
+    ms_per_step = elapsed_ms / args.steps
+    value = n * world / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API, host buffers (pinned), copies inside
+    e2e = None
+    if not args.no_e2e:
+        k = max(3, min(args.steps, 10))
+        h_codes = torch.empty((n, 8), dtype=torch.int16, pin_memory=True)
+        h_x = torch.empty((n, 512), dtype=torch.float32, pin_memory=True) if do_dec else None
+        if do_enc:
+            h_z = torch.empty(z.shape, dtype=z.dtype, pin_memory=True)
+            h_z.copy_(z)
+            bi = h_z.numel() * h_z.element_size()
+        else:
+            h_in = torch.empty(codes.shape, dtype=codes.dtype, pin_memory=True)
+            h_in.copy_(codes)
+            bi = h_in.numel() * h_in.element_size()
+        bo = (h_codes.numel() * 2 if do_enc else 0) + (h_x.numel() * 4 if do_dec else 0)
+
+        def e2e_step():
+            if do_enc:
+                z.copy_(h_z, non_blocking=True)
+                q.encode(z, out=codes, stream=stream)
+                h_codes.copy_(codes, non_blocking=True)
+            else:
+                codes.copy_(h_in, non_blocking=True)
+            if do_dec:
+                q.decode(codes, out=x, stream=stream)
+                h_x.copy_(x, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if dist:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(k):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = a.elapsed_time(b) / k
+        if dist:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": n * world / (e_ms / 1e3), "unit": "frames/s", "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": e_ms, "steps": k}
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return None
+
+    peaks = load_peaks()
+    kernels = []
+    lat_bytes = 2048 if work.get("dtype", "f32") == "f32" else 1024
+    if do_enc:
+        tf = ENC_FLOP * n / (enc_avg / 1e3) / 1e12
+        kernels.append({
+            "kernel": "encode call (k_encode_tc + full-scan fallback)", "bound": "tensor",
+            "achieved": tf, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops_sustained"], "traffic": None, "ms": enc_avg,
+            "algorithmic": f"{ENC_FLOP} FLOP/frame x {n} frames; HBM {lat_bytes + 16} B/frame",
+            "hbm_gbs": (lat_bytes + 16) * n / (enc_avg / 1e3) / 1e9})
+    if do_dec:
+        gbs = DEC_BYTES * n / (dec_avg / 1e3) / 1e9
+        kernels.append({
+            "kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms": dec_avg,
+            "algorithmic": f"{DEC_BYTES} B/frame x {n} frames (codes in, fp32 latents out)"})
+    dominant = kernels[0]
+    roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = dominant["kernel"]
+    roofline["peak_source"] = (f"{peaks['source']} "
+                               f"{'bf16_tflops_sustained' if dominant['bound'] == 'tensor' else 'hbm_gbs'}")
+    launches_per_step = (2 if do_enc else 0) + (1 if do_dec else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 products, f32 accumulate/re-score", "data": "synthetic",
+        "config": {"workload": f"{name}: {WORKLOADS[name]}" + (
+                       f" (reduced to {n} frames)" if args.frames else ""), "frames_per_gpu": n,
+                   "latent_dtype": work.get("dtype"), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (not re-read from L2 between steps)"},
+        "realtime_streams": value / FRAME_HZ,
+        "roofline": roofline, "kernels": kernels,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(), "status": status, "e2e": e2e,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(work, name)
+    if dist:
+        dist.destroy_process_group()
+    return line
+
+
+def run_streaming(args):
+    """Per-call device latency of encode_step for B in {1, 16, 128, 1024}, 1000 calls each
+    (L2 flushed between calls when the inputs would fit in it)."""
+    import torch
+    import split_residual_vector_b200 as pkg
+    device = torch.device("cuda", 0)
+    out = {}
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)  # 256 MiB > L2
+    for B in (1, 16, 128, 1024):
+        model, frames = synth.streaming_step(B, calls=args.calls)
+        q = pkg.Quantizer(torch.from_numpy(model.C).to(device),
+                          torch.from_numpy(model.W_in).to(device),
+                          torch.from_numpy(model.W_out).to(device))
+        f = torch.from_numpy(frames).to(device)
+        codes = torch.empty((B, 8), dtype=torch.int16, device=device)
+        stream = torch.cuda.current_stream(device)
+        for i in range(5):
+            q.encode_step(f[i], out=codes, stream=stream)
+        need_flush = frames.nbytes < (256 << 20)
+        times = []
+        for i in range(args.calls):
+            if need_flush:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            q.encode_step(f[i], out=codes, stream=stream)
+            b.record(stream)
+            times.append((a, b))
+        torch.cuda.synchronize(device)
+        ms = sorted(a.elapsed_time(b) for a, b in times)
+        out[B] = {"median_us": 1e3 * ms[len(ms) // 2], "p99_us": 1e3 * ms[int(0.99 * len(ms))],
+                  "frames_per_s": B / (ms[len(ms) // 2] / 1e3), "l2_flushed": need_flush}
+        q.close()
+    return {"metric": METRIC, "workload": f"streaming: {WORKLOADS['streaming']}",
+            "calls": args.calls, "per_batch": out}
+
+
+# --------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    """The float64 oracle on the host cores, each step a bounded sample of the workload."""
+    import oracle
+    name = args.workload
+    work = make_workload(name, 0)
+    m = work["model"]
+
+    def one(nf):
+        if name in ("offline_batch", "bulk_tokenization"):
+            c, _, _ = oracle.encode(work["z"][:nf], m.W_in, m.C)
+            if name == "offline_batch":
+                oracle.decode(c, m.C, m.W_out)
+        else:
+            oracle.decode(work["codes"][:nf], m.C, m.W_out)
+
+    t0 = time.perf_counter()
+    one(32)
+    per_frame = (time.perf_counter() - t0) / 32
+    budget = 120.0 / (args.steps + args.warmup)  # whole run within ~2 minutes
+    nf = int(max(8, min(work["frames"], budget / max(per_frame, 1e-9))))
+    for _ in range(args.warmup):
+        one(nf)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one(nf)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = nf / dt
+    cores = oracle.threads(0)
+    sample = f"first {nf} frames of {name} per step, float64 oracle"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "frames/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{name}: {WORKLOADS[name]}", "sample_frames": nf},
+            "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="offline_batch", choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--calls", type=int, default=1000, help="streaming workload: calls per B")
+    ap.add_argument("--frames", type=int, default=None,
+                    help="shrink the workload (for profiler captures); default: full size")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload == "streaming":
+        if rank == 0:
+            print(json.dumps(run_streaming(args)), flush=True)
+        return
+    line = run_ours(args, rank, world, local_rank)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -139,7 +139,7 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (e == cudaSuccess) e = dalloc(&t.Win_hi, (size_t)kD * kDin);
     if (e == cudaSuccess) e = dalloc(&t.Win_lo, (size_t)kD * kDin);
     if (e == cudaSuccess) e = dalloc(&t.cnorm, (size_t)kQ * kK);
-    if (e == cudaSuccess) e = dalloc(&t.cbound, (size_t)2 * kQ);
+    if (e == cudaSuccess) e = dalloc(&t.cbound, (size_t)4 * kQ);
     if (e == cudaSuccess) e = dalloc(&t.P, (size_t)kQ * kK * kDin);
     if (e == cudaSuccess) e = dalloc(&t.err, 1);
     if (e == cudaSuccess) e = dalloc(&t.rescan_count, 1);

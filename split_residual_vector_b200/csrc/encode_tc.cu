@@ -14,8 +14,9 @@
 //      streamed by TMA into a shared-memory ring; accumulators double-buffered
 //      in TMEM columns [256, 512)). The epilogue keeps a sorted top-8 per row.
 //   3. certified pick: with E a rigorous bound on |bf16 score - exact score|
-//      (from ||r||, max ||c|| of the codebook and the bf16 / fp32 rounding
-//      units), every codeword outside the top-8 is ruled out when
+//      (from ||r||, this row's bf16 rounding residual ||bf16(r) - r||, and the
+//      codebook's max ||c|| and max ||bf16(c) - c||), every codeword outside
+//      the top-8 is ruled out when
 //      s_8 > s_1 + 2E; the candidates within s_1 + 2E are re-scored in float32
 //      (||c||^2 - 2 r.c with r read from TMEM and c from the float32
 //      codebook); a single candidate needs no re-score. If the top-8 cannot be
@@ -54,11 +55,17 @@ constexpr int kThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
 
-// bound coefficients (see header comment): bf16 rounding of both operands
-// (2 u + u^2, u = 2^-9), fp32 accumulation of 256 products (<= 2^-15 of the
-// absolute sum), times 2 for the -2 r.c, plus slack.
-constexpr float kBoundDot = 0.0080f;
-constexpr float kBoundNorm = 4.8e-7f;   // > 2^-21: fp32 rounding of ||c||^2 and of the score
+// Candidate bound. With e_r = bf16(r) - r and e_c = bf16(c) - c,
+//   bf16(r).bf16(c) - r.c = r.e_c + e_r.c + e_r.e_c,
+// so by Cauchy-Schwarz |error of the product sum| <= ||r|| ||e_c|| + ||e_r|| ||c||
+// + ||e_r|| ||e_c||, using the exact ||e_r|| of this row and the codebook's
+// max ||c||, max ||e_c||. The tensor core's float32 accumulation of 256
+// products adds at most 256 * 2^-23 of the absolute sum (taken as 2^-14 of
+// ||bf16(r)|| ||bf16(c)||, twice the need), and the float32 score
+// ||c||^2 - 2 acc rounds once more (2^-21 of its magnitude, with slack).
+// E bounds |bf16 score - exact score| for every codeword.
+constexpr float kAccRel = 6.103515625e-05f;    // 2^-14
+constexpr float kScoreRel = 4.76837158203125e-07f;  // 2^-21
 
 struct Bars {
     uint64_t full[STAGES], empty[STAGES];
@@ -315,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = ewait(&bars->yfull, tile_iter & 1);
             if (!ok) break;
             tc_fence_after();
-            float nr2 = 0.f;
+            float nr2 = 0.f, ner2 = 0.f;  // ||r||^2 and ||bf16(r) - r||^2 of this row
             for (int ch = 0; ch < kD / 32; ++ch) {
                 uint32_t v[32];
                 tmem_ld32(trow + ch * 32, v);
@@ -336,6 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nr2 = fmaf(a, a, nr2);
                     nr2 = fmaf(b, b, nr2);
                     pk[i] = pack_bf16x2(a, b);
+                    const float ea = bf16_lo_to_f32(pk[i]) - a, eb = bf16_hi_to_f32(pk[i]) - b;
+                    ner2 = fmaf(ea, ea, ner2);
+                    ner2 = fmaf(eb, eb, ner2);
                 }
                 uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
 #pragma unroll
@@ -397,9 +407,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 // ---- certified window and float32 re-score
-                const float cmax = __ldg(cbound + 2 * l), cnmax = __ldg(cbound + 2 * l + 1);
-                const float nr = sqrtf(nr2) * 1.0001f;
-                const float E = nr * cmax * kBoundDot + cnmax * kBoundNorm;
+                const float cmax = __ldg(cbound + 4 * l), cnmax = __ldg(cbound + 4 * l + 1);
+                const float ecmax = __ldg(cbound + 4 * l + 2);
+                const float nr = sqrtf(nr2) * 1.0001f, ner = sqrtf(ner2) * 1.0001f;
+                const float dot_err = nr * ecmax + ner * cmax + ner * ecmax +
+                                      kAccRel * (nr + ner) * (cmax + ecmax);
+                const float E = 2.f * dot_err * 1.0001f +
+                                kScoreRel * (cnmax + 2.f * (nr + ner) * (cmax + ecmax));
                 const float thr = ts[0] + 2.f * E;
                 int m = 0;
 #pragma unroll
@@ -457,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++aecnt;
                     if (!ok) break;
                     nr2 = 0.f;
+                    ner2 = 0.f;
                     const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD);
                     for (int ch = 0; ch < kD / 32; ++ch) {
                         uint32_t v[32];
@@ -481,6 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             nr2 = fmaf(a, a, nr2);
                             nr2 = fmaf(b, b, nr2);
                             pk[i] = pack_bf16x2(a, b);
+                            const float ea = bf16_lo_to_f32(pk[i]) - a;
+                            const float eb = bf16_hi_to_f32(pk[i]) - b;
+                            ner2 = fmaf(ea, ea, ner2);
+                            ner2 = fmaf(eb, eb, ner2);
                         }
                         uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
 #pragma unroll

@@ -29,7 +29,7 @@ struct Tables {
     __nv_bfloat16* Win_hi = nullptr;  // [D][Din] bf16(W_in)
     __nv_bfloat16* Win_lo = nullptr;  // [D][Din] bf16(W_in - Win_hi)
     float* cnorm = nullptr;           // [Q][K] ||c||^2 (float64 sum, rounded)
-    float* cbound = nullptr;          // [Q][2]: max ||c|| (rounded up), max ||c||^2
+    float* cbound = nullptr;          // [Q][4]: max ||c||, max ||c||^2, max ||bf16(c) - c||, 0 (rounded up)
     float* P = nullptr;               // [Q][K][Din] W_out . c (float64 sum, rounded): decode rows
     // device state
     int* err = nullptr;               // error bits (MIMI_DEV_ERR_*)

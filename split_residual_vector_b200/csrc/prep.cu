@@ -16,22 +16,32 @@ __global__ void k_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restri
 }
 
 // One warp per codeword: ||c||^2 in float64, rounded to float32; and the
-// per-codebook maxima of ||c|| and ||c||^2, rounded up, for the candidate bound.
+// per-codebook maxima, rounded up, that the candidate bound needs:
+// cbound[4q + 0] = max ||c||, [4q + 1] = max ||c||^2, [4q + 2] = max ||bf16(c) - c||.
 __global__ void k_norms(const float* __restrict__ C, float* __restrict__ cnorm,
                         float* __restrict__ cbound) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= kQ * kK) return;
     const float* c = C + (size_t)warp * kD;
-    double s = 0.0;
-    for (int i = lane; i < kD; i += 32) s += (double)c[i] * (double)c[i];
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    double s = 0.0, e = 0.0;
+    for (int i = lane; i < kD; i += 32) {
+        const double v = (double)c[i];
+        const double d = (double)__bfloat162float(__float2bfloat16_rn(c[i])) - v;
+        s += v * v;
+        e += d * d;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
     if (lane == 0) {
         cnorm[warp] = (float)s;
         const int q = warp / kK;
-        // positive floats order like their bit patterns
-        atomicMax(reinterpret_cast<int*>(&cbound[2 * q]), __float_as_int(__double2float_ru(sqrt(s))));
-        atomicMax(reinterpret_cast<int*>(&cbound[2 * q + 1]), __float_as_int(__double2float_ru(s)));
+        // non-negative floats order like their bit patterns
+        atomicMax(reinterpret_cast<int*>(&cbound[4 * q + 0]), __float_as_int(__double2float_ru(sqrt(s))));
+        atomicMax(reinterpret_cast<int*>(&cbound[4 * q + 1]), __float_as_int(__double2float_ru(s)));
+        atomicMax(reinterpret_cast<int*>(&cbound[4 * q + 2]), __float_as_int(__double2float_ru(sqrt(e))));
     }
 }
 
@@ -93,7 +103,7 @@ __global__ void __launch_bounds__(256) k_decode_table(const float* __restrict__ 
 cudaError_t prep_tables(Tables& t, const float* W_out, cudaStream_t s) {
     const int64_t nC = (int64_t)kQ * kK * kD;
     k_to_bf16<<<592, 256, 0, s>>>(t.C32, t.Cbf, nC);
-    cudaError_t e = cudaMemsetAsync(t.cbound, 0, sizeof(float) * 2 * kQ, s);
+    cudaError_t e = cudaMemsetAsync(t.cbound, 0, sizeof(float) * 4 * kQ, s);
     if (e != cudaSuccess) return e;
     k_norms<<<(kQ * kK * 32 + 255) / 256, 256, 0, s>>>(t.C32, t.cnorm, t.cbound);
     k_split_win<<<(kD * kDin + 255) / 256, 256, 0, s>>>(t.Win32, t.Win_hi, t.Win_lo, t.WinT32);
