@@ -47,11 +47,16 @@ constexpr int STAGES = 8;
 constexpr int STAGE_BYTES = BN * BK * 2;        // 16 KiB
 constexpr int A_CHUNK_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int RING_OFF = 0;
-constexpr int A_OFF = STAGES * STAGE_BYTES;     // 128 KiB
-constexpr int BAR_OFF = A_OFF + KCH * A_CHUNK_BYTES;  // 192 KiB
-constexpr int SMEM_BYTES = BAR_OFF + 1024 + 1024;     // barriers, slack for 1 KiB alignment
+constexpr int A_OFF = STAGES * STAGE_BYTES;             // 128 KiB
+constexpr int X_OFF = A_OFF + KCH * A_CHUNK_BYTES;      // 192 KiB: epilogue exchange area
+constexpr int XKEYS_OFF = X_OFF;                        // [BM][TOPK] float keys
+constexpr int XWIN_OFF = XKEYS_OFF + BM * 8 * 4;        // [BM] int winners
+constexpr int XNORM_OFF = XWIN_OFF + BM * 4;            // [2][BM][2] partial norms
+constexpr int BAR_OFF = XNORM_OFF + 2 * BM * 2 * 4;
+constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;        // barriers, slack for 1 KiB alignment
 constexpr int TOPK = 8;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;            // two per TMEM lane quarter: column halves
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
 
@@ -64,30 +69,45 @@ constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
 // ||bf16(r)|| ||bf16(c)||, twice the need), and the float32 score
 // ||c||^2 - 2 acc rounds once more (2^-21 of its magnitude, with slack).
 // E bounds |bf16 score - exact score| for every codeword.
-constexpr float kAccRel = 6.103515625e-05f;    // 2^-14
+constexpr float kAccRel = 6.103515625e-05f;         // 2^-14
 constexpr float kScoreRel = 4.76837158203125e-07f;  // 2^-21
+
+// Candidate keys: a float32 score whose low 11 mantissa bits are replaced by
+// the codeword index, so that one min/max orders (score, index) pairs and the
+// index travels with the score. The replacement moves the value by less than
+// 2^-12 of its magnitude; every comparison that must be rigorous widens by
+// key_slack(x) = 2^-11 |x|, which covers it.
+__device__ __forceinline__ float make_key(float s, int idx) {
+    return __int_as_float((__float_as_int(s) & ~0x7FF) | idx);
+}
+__device__ __forceinline__ int key_index(float k) { return __float_as_int(k) & 0x7FF; }
+__device__ __forceinline__ float key_slack(float k) { return fabsf(k) * 4.8828125e-4f; }
 
 struct Bars {
     uint64_t full[STAGES], empty[STAGES];
     uint64_t zfull[2], zempty[2];
     uint64_t yfull, afull, aempty, drain;
     uint64_t tfull[2], tempty[2];
+    uint64_t ebar;          // epilogue-wide barrier (all epilogue threads arrive)
     uint32_t tmem_base;
     int abort;
 };
 
-__device__ __forceinline__ void insert_top8(float (&ts)[TOPK], int (&ti)[TOPK], float s, int k) {
+// Insert key k into the ascending list ts[0..7] (the largest falls off).
+__device__ __forceinline__ void insert_key(float (&ts)[TOPK], float k) {
 #pragma unroll
     for (int p = 0; p < TOPK; ++p) {
-        if (s < ts[p]) {
-            const float ft = ts[p];
-            const int it = ti[p];
-            ts[p] = s;
-            ti[p] = k;
-            s = ft;
-            k = it;
-        }
+        const float lo = fminf(ts[p], k);
+        k = fmaxf(ts[p], k);
+        ts[p] = lo;
     }
+}
+
+// Threshold above which a raw score can be dropped: it is outside the window
+// of the current best (and the best only improves), or it would fall off the
+// full list at once.
+__device__ __forceinline__ float scan_threshold(const float (&ts)[TOPK], float twoE) {
+    return fminf(ts[TOPK - 1] + key_slack(ts[TOPK - 1]), ts[0] + key_slack(ts[0]) + twoE);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -119,15 +139,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->zfull[b], 4);
+            mbar_init(&bars->zfull[b], kEpiWarps);
             mbar_init(&bars->zempty[b], 1);
             mbar_init(&bars->tfull[b], 1);
-            mbar_init(&bars->tempty[b], 4);
+            mbar_init(&bars->tempty[b], kEpiWarps);
         }
         mbar_init(&bars->yfull, 1);
-        mbar_init(&bars->afull, 4);
+        mbar_init(&bars->afull, kEpiWarps);
         mbar_init(&bars->aempty, 1);
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->ebar, 32 * kEpiWarps);
         bars->abort = 0;
         fence_mbar_init();
     }
@@ -253,9 +274,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Eight warps. Warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows);
+        // the two warps of a lane quarter split every 128-column score tile
+        // (half h takes columns 64 h .. + 63) and the 256 dimensions of r
+        // (half h owns dimensions 128 h .. + 127). Each thread keeps a sorted
+        // list of its half's 8 best keys; the halves merge at the end of a level.
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
+        int* xwin = reinterpret_cast<int*>(smem + XWIN_OFF);
+        float* xnorm = reinterpret_cast<float*>(smem + XNORM_OFF);
         uint32_t zuse[2] = {0, 0}, aecnt = 0, tcnt = 0, tile_iter = 0;
         bool ok = true;
         unsigned long long done = 0;
@@ -265,16 +295,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool r = mbar_wait(bar, parity, abort, err);
             return __all_sync(0xffffffffu, r) != 0;
         };
+        // Pack this half's 128 dimensions of r (TMEM chunks 4h..4h+3, held in
+        // v by the caller one chunk at a time) into the A operand and its norms.
+        auto write_a_chunk = [&](int ch, const uint32_t (&v)[32], float& nr2, float& ner2) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+                nr2 = fmaf(a, a, nr2);
+                nr2 = fmaf(b, b, nr2);
+                pk[i] = pack_bf16x2(a, b);
+                const float ea = bf16_lo_to_f32(pk[i]) - a, eb = bf16_hi_to_f32(pk[i]) - b;
+                ner2 = fmaf(ea, ea, ner2);
+                ner2 = fmaf(eb, eb, ner2);
+            }
+            uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                *reinterpret_cast<uint4*>(dst + sw128_offset(row, (ch & 1) * 4 + p)) =
+                    make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
+        };
+        // Barrier over the epilogue threads on an mbarrier, so that the wait is
+        // bounded and gives way when another warp has aborted.
+        uint32_t ephase = 0;
+        auto esync = [&]() {
+            mbar_arrive(&bars->ebar);
+            const bool r = mbar_wait(&bars->ebar, ephase & 1, abort, err);
+            ++ephase;
+            return __all_sync(0xffffffffu, r) != 0;
+        };
+        // Both halves publish their partial norms; both read back the same sum.
+        auto combine_norms = [&](float& nr2, float& ner2) {
+            xnorm[(half * BM + row) * 2 + 0] = nr2;
+            xnorm[(half * BM + row) * 2 + 1] = ner2;
+            if (!esync()) return false;
+            nr2 = xnorm[row * 2 + 0] + xnorm[(BM + row) * 2 + 0];
+            ner2 = xnorm[row * 2 + 1] + xnorm[(BM + row) * 2 + 1];
+            return true;
+        };
+
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tile_iter) {
             const int64_t frame = tile * BM + row;
             const bool valid = frame < n;
-            // A region is z staging now: wait until the previous tile's level-7 MMAs are done
+            // the A region is z staging now: wait for the previous tile's last MMAs
             if (tile_iter > 0 && n_q > 0) {
                 ok = ewait(&bars->aempty, aecnt & 1);
                 ++aecnt;
                 if (!ok) break;
             }
-            // ---- stage z (split into bf16 hi / lo) for the projection
+            // ---- stage z (bf16 hi / lo split) for the projection; this half
+            //      writes pieces 4h..4h+3 (32 elements) of each 64-wide K chunk
             for (int kc = 0; kc < PKCH && ok; ++kc) {
                 const int zb = kc & 1;
                 if (zuse[zb] > 0) {
@@ -284,33 +354,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++zuse[zb];
                 uint8_t* zhi = smem + A_OFF + zb * 2 * A_CHUNK_BYTES;
                 uint8_t* zlo = zhi + A_CHUNK_BYTES;
+                const int e0 = kc * BK + half * 32;
                 if (f32_in) {
-                    const float4* src =
-                        reinterpret_cast<const float4*>(static_cast<const float*>(z) +
-                                                        (valid ? frame : 0) * kDin + kc * BK);
+                    const float4* src = reinterpret_cast<const float4*>(
+                        static_cast<const float*>(z) + (valid ? frame : 0) * kDin + e0);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        float4 u = valid ? __ldg(src + 2 * p) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        float4 v = valid ? __ldg(src + 2 * p + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int p = 0; p < 4; ++p) {
+                        const float4 u = valid ? __ldg(src + 2 * p) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        const float4 w = valid ? __ldg(src + 2 * p + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
                         uint4 h, lo;
                         h.x = pack_bf16x2(u.x, u.y);
                         h.y = pack_bf16x2(u.z, u.w);
-                        h.z = pack_bf16x2(v.x, v.y);
-                        h.w = pack_bf16x2(v.z, v.w);
+                        h.z = pack_bf16x2(w.x, w.y);
+                        h.w = pack_bf16x2(w.z, w.w);
                         lo.x = pack_bf16x2(u.x - bf16_lo_to_f32(h.x), u.y - bf16_hi_to_f32(h.x));
                         lo.y = pack_bf16x2(u.z - bf16_lo_to_f32(h.y), u.w - bf16_hi_to_f32(h.y));
-                        lo.z = pack_bf16x2(v.x - bf16_lo_to_f32(h.z), v.y - bf16_hi_to_f32(h.z));
-                        lo.w = pack_bf16x2(v.z - bf16_lo_to_f32(h.w), v.w - bf16_hi_to_f32(h.w));
-                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, p)) = h;
-                        *reinterpret_cast<uint4*>(zlo + sw128_offset(row, p)) = lo;
+                        lo.z = pack_bf16x2(w.x - bf16_lo_to_f32(h.z), w.y - bf16_hi_to_f32(h.z));
+                        lo.w = pack_bf16x2(w.z - bf16_lo_to_f32(h.w), w.w - bf16_hi_to_f32(h.w));
+                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, half * 4 + p)) = h;
+                        *reinterpret_cast<uint4*>(zlo + sw128_offset(row, half * 4 + p)) = lo;
                     }
                 } else {
                     const uint4* src = reinterpret_cast<const uint4*>(
-                        static_cast<const uint16_t*>(z) + (valid ? frame : 0) * kDin + kc * BK);
+                        static_cast<const uint16_t*>(z) + (valid ? frame : 0) * kDin + e0);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
+                    for (int p = 0; p < 4; ++p) {
                         const uint4 h = valid ? __ldg(src + p) : make_uint4(0u, 0u, 0u, 0u);
-                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, p)) = h;
+                        *reinterpret_cast<uint4*>(zhi + sw128_offset(row, half * 4 + p)) = h;
                     }
                 }
                 fence_proxy_async_smem();
@@ -318,12 +388,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&bars->zfull[zb]);
             }
             if (!ok) break;
-            // ---- y from TMEM: norm and the bf16 A operand of levels 0 and 1
+            // ---- y from TMEM: this half's 128 dimensions -> A operand (levels 0, 1), norms
             ok = ewait(&bars->yfull, tile_iter & 1);
             if (!ok) break;
             tc_fence_after();
             float nr2 = 0.f, ner2 = 0.f;  // ||r||^2 and ||bf16(r) - r||^2 of this row
-            for (int ch = 0; ch < kD / 32; ++ch) {
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int ch = half * 4 + c4;
                 uint32_t v[32];
                 tmem_ld32(trow + ch * 32, v);
                 tmem_wait_ld();
@@ -335,145 +406,165 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               __uint_as_float(v[4 * q4 + 2]),
                                               __uint_as_float(v[4 * q4 + 3]));
                 }
-                if (n_q == 0) continue;
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
-                    nr2 = fmaf(a, a, nr2);
-                    nr2 = fmaf(b, b, nr2);
-                    pk[i] = pack_bf16x2(a, b);
-                    const float ea = bf16_lo_to_f32(pk[i]) - a, eb = bf16_hi_to_f32(pk[i]) - b;
-                    ner2 = fmaf(ea, ea, ner2);
-                    ner2 = fmaf(eb, eb, ner2);
-                }
-                uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(row, (ch & 1) * 4 + p)) =
-                        make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
+                if (n_q > 0) write_a_chunk(ch, v, nr2, ner2);
             }
             tc_fence_before();
             if (n_q == 0) continue;  // projection only: y has been written out
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->afull);
+            ok = combine_norms(nr2, ner2);
+            if (!ok) break;
 
             int win_codes[kQ];
             bool flagged = false;
             for (int l = 0; l < n_q && ok; ++l) {
-                float ts[TOPK];
-                int ti[TOPK];
-#pragma unroll
-                for (int p = 0; p < TOPK; ++p) {
-                    ts[p] = __int_as_float(0x7f800000);
-                    ti[p] = 0x7fffffff;
-                }
                 const float* cn = cnorm + (size_t)l * kK;
-                // ---- scan the 16 score tiles of this codebook
+                const float* book = C32 + (size_t)l * kK * kD;
+                const float4 cb = __ldg(reinterpret_cast<const float4*>(cbound) + l);
+                const float cmax = cb.x, cnmax = cb.y, ecmax = cb.z;
+                const float nr = sqrtf(nr2) * 1.0001f, ner = sqrtf(ner2) * 1.0001f;
+                const float dot_err = nr * ecmax + ner * cmax + ner * ecmax +
+                                      kAccRel * (nr + ner) * (cmax + ecmax);
+                const float E = 2.f * dot_err * 1.0001f +
+                                kScoreRel * (cnmax + 2.f * (nr + ner) * (cmax + ecmax));
+                const float twoE = 2.f * E;
+                float ts[TOPK];
+#pragma unroll
+                for (int p = 0; p < TOPK; ++p) ts[p] = __int_as_float(0x7f800000);
+                float thr = __int_as_float(0x7f800000);
+                // ---- scan this half of the 16 score tiles of the codebook
                 for (int nt = 0; nt < NT; ++nt) {
                     const int bsel = tcnt & 1;
                     ok = ewait(&bars->tfull[bsel], (tcnt >> 1) & 1);
                     ++tcnt;
                     if (!ok) break;
                     tc_fence_after();
-                    for (int ch = 0; ch < BN / 32; ++ch) {
+#pragma unroll 1
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const int ch = half * 2 + c2;
                         uint32_t v[32];
                         tmem_ld32(trow + TMEM_SCORE + bsel * BN + ch * 32, v);
                         tmem_wait_ld();
-                        if (ch == BN / 32 - 1) {
+                        if (c2 == 1) {
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
                         }
                         const int k0 = nt * BN + ch * 32;
                         const float4* cn4 = reinterpret_cast<const float4*>(cn + k0);
+                        float sc[32];
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4) {
                             const float4 c = __ldg(cn4 + q4);
-                            const float s0 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 0]), c.x);
-                            const float s1 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 1]), c.y);
-                            const float s2 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 2]), c.z);
-                            const float s3 = fmaf(-2.f, __uint_as_float(v[4 * q4 + 3]), c.w);
-                            const float m = fminf(fminf(s0, s1), fminf(s2, s3));
-                            if (m < ts[TOPK - 1]) {
-                                insert_top8(ts, ti, s0, k0 + 4 * q4 + 0);
-                                insert_top8(ts, ti, s1, k0 + 4 * q4 + 1);
-                                insert_top8(ts, ti, s2, k0 + 4 * q4 + 2);
-                                insert_top8(ts, ti, s3, k0 + 4 * q4 + 3);
+                            sc[4 * q4 + 0] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 0]), c.x);
+                            sc[4 * q4 + 1] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 1]), c.y);
+                            sc[4 * q4 + 2] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 2]), c.z);
+                            sc[4 * q4 + 3] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 3]), c.w);
+                        }
+                        float g[8];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            g[q4] = fminf(fmin3(sc[4 * q4], sc[4 * q4 + 1], sc[4 * q4 + 2]),
+                                          sc[4 * q4 + 3]);
+                        const float cm = fminf(fmin3(g[0], g[1], g[2]), fmin3(g[3], g[4], fmin3(g[5], g[6], g[7])));
+                        // the chunk minimum tightens the window before its groups are scanned
+                        thr = fminf(thr, cm + key_slack(cm) + twoE);
+                        if (cm <= thr) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4) {
+                                if (g[q4] <= thr) {
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const float sv = sc[4 * q4 + e];
+                                        if (sv <= thr) {
+                                            insert_key(ts, make_key(sv, k0 + 4 * q4 + e));
+                                            thr = scan_threshold(ts, twoE);
+                                        }
+                                    }
+                                }
                             }
                         }
                     }
                 }
                 if (!ok) break;
-                // ---- certified window and float32 re-score
-                const float cmax = __ldg(cbound + 4 * l), cnmax = __ldg(cbound + 4 * l + 1);
-                const float ecmax = __ldg(cbound + 4 * l + 2);
-                const float nr = sqrtf(nr2) * 1.0001f, ner = sqrtf(ner2) * 1.0001f;
-                const float dot_err = nr * ecmax + ner * cmax + ner * ecmax +
-                                      kAccRel * (nr + ner) * (cmax + ecmax);
-                const float E = 2.f * dot_err * 1.0001f +
-                                kScoreRel * (cnmax + 2.f * (nr + ner) * (cmax + ecmax));
-                const float thr = ts[0] + 2.f * E;
-                int m = 0;
+                // ---- merge the halves; certified window; float32 re-score
+                if (half == 1) {
 #pragma unroll
-                for (int p = 0; p < TOPK; ++p) m += (ts[p] <= thr) ? 1 : 0;
-                if (valid && !(ts[TOPK - 1] > thr) && !flagged) {
-                    flagged = true;
-                    const int slot = atomicAdd(rescan_count, 1);
-                    if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
+                    for (int p = 0; p < TOPK; ++p) xkeys[row * TOPK + p] = ts[p];
                 }
-                const float* book = C32 + (size_t)l * kK * kD;
-                int win = ti[0];
-                if (__any_sync(0xffffffffu, m > 1)) {
-                    float dot[TOPK];
+                ok = esync();
+                if (!ok) break;
+                int win = 0;
+                if (half == 0) {
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
-                    for (int ch = 0; ch < kD / 32; ++ch) {
-                        uint32_t v[32];
-                        tmem_ld32(trow + ch * 32, v);
-                        tmem_wait_ld();
+                    for (int p = 0; p < TOPK; ++p) insert_key(ts, xkeys[row * TOPK + p]);
+                    const float wthr = ts[0] + key_slack(ts[0]) + twoE;
+                    int m = 0;
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) m += (ts[p] - key_slack(ts[p]) <= wthr) ? 1 : 0;
+                    const bool certified = ts[TOPK - 1] - key_slack(ts[TOPK - 1]) > wthr;
+                    if (valid && !certified && !flagged) {
+                        flagged = true;
+                        const int slot = atomicAdd(rescan_count, 1);
+                        if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
+                    }
+                    win = key_index(ts[0]);
+                    if (__any_sync(0xffffffffu, m > 1)) {
+                        float dot[TOPK];
+#pragma unroll
+                        for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
+                        for (int ch = 0; ch < kD / 32; ++ch) {
+                            uint32_t v[32];
+                            tmem_ld32(trow + ch * 32, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int p = 0; p < TOPK; ++p) {
+                                if (p < m) {
+                                    const float4* c4 = reinterpret_cast<const float4*>(
+                                        book + (size_t)key_index(ts[p]) * kD + ch * 32);
+                                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                                    for (int q4 = 0; q4 < 8; ++q4) {
+                                        const float4 c = __ldg(c4 + q4);
+                                        a0 = fmaf(__uint_as_float(v[4 * q4 + 0]), c.x, a0);
+                                        a1 = fmaf(__uint_as_float(v[4 * q4 + 1]), c.y, a1);
+                                        a0 = fmaf(__uint_as_float(v[4 * q4 + 2]), c.z, a0);
+                                        a1 = fmaf(__uint_as_float(v[4 * q4 + 3]), c.w, a1);
+                                    }
+                                    dot[p] += a0 + a1;
+                                }
+                            }
+                        }
+                        float best = __int_as_float(0x7f800000);
 #pragma unroll
                         for (int p = 0; p < TOPK; ++p) {
                             if (p < m) {
-                                const float4* c4 = reinterpret_cast<const float4*>(
-                                    book + (size_t)ti[p] * kD + ch * 32);
-                                float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                                for (int q4 = 0; q4 < 8; ++q4) {
-                                    const float4 c = __ldg(c4 + q4);
-                                    a0 = fmaf(__uint_as_float(v[4 * q4 + 0]), c.x, a0);
-                                    a1 = fmaf(__uint_as_float(v[4 * q4 + 1]), c.y, a1);
-                                    a0 = fmaf(__uint_as_float(v[4 * q4 + 2]), c.z, a0);
-                                    a1 = fmaf(__uint_as_float(v[4 * q4 + 3]), c.w, a1);
+                                const int k = key_index(ts[p]);
+                                const float e = fmaf(-2.f, dot[p], __ldg(cn + k));
+                                if (e < best || (e == best && k < win)) {
+                                    best = e;
+                                    win = k;
                                 }
-                                dot[p] += a0 + a1;
                             }
                         }
                     }
-                    float best = __int_as_float(0x7f800000);
-#pragma unroll
-                    for (int p = 0; p < TOPK; ++p) {
-                        if (p < m) {
-                            const float e = fmaf(-2.f, dot[p], __ldg(cn + ti[p]));
-                            if (e < best || (e == best && ti[p] < win)) {
-                                best = e;
-                                win = ti[p];
-                            }
-                        }
-                    }
+                    win_codes[l] = win;
+                    xwin[row] = win;
                 }
-                if (win < 0 || win >= kK) win = 0;  // only reachable with NaN / Inf inputs
-                win_codes[l] = win;
-                // ---- residual update r -= c_win (levels feeding another level)
+                // ---- residual update r -= c_win for the next level, split by halves
                 if (updates_after(l)) {
+                    ok = esync();
+                    if (!ok) break;
+                    win = xwin[row];
                     ok = ewait(&bars->aempty, aecnt & 1);
                     ++aecnt;
                     if (!ok) break;
                     nr2 = 0.f;
                     ner2 = 0.f;
                     const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD);
-                    for (int ch = 0; ch < kD / 32; ++ch) {
+                    for (int c4i = 0; c4i < 4; ++c4i) {
+                        const int ch = half * 4 + c4i;
                         uint32_t v[32];
                         tmem_ld32(trow + ch * 32, v);
                         float4 c[8];
@@ -488,44 +579,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                             v[4 * q4 + 3] = __float_as_uint(__uint_as_float(v[4 * q4 + 3]) - c[q4].w);
                         }
                         tmem_st32(trow + ch * 32, v);
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float a = __uint_as_float(v[2 * i]);
-                            const float b = __uint_as_float(v[2 * i + 1]);
-                            nr2 = fmaf(a, a, nr2);
-                            nr2 = fmaf(b, b, nr2);
-                            pk[i] = pack_bf16x2(a, b);
-                            const float ea = bf16_lo_to_f32(pk[i]) - a;
-                            const float eb = bf16_hi_to_f32(pk[i]) - b;
-                            ner2 = fmaf(ea, ea, ner2);
-                            ner2 = fmaf(eb, eb, ner2);
-                        }
-                        uint8_t* dst = smem + A_OFF + (ch >> 1) * A_CHUNK_BYTES;
-#pragma unroll
-                        for (int p = 0; p < 4; ++p)
-                            *reinterpret_cast<uint4*>(dst + sw128_offset(row, (ch & 1) * 4 + p)) =
-                                make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
+                        write_a_chunk(ch, v, nr2, ner2);
                     }
                     tmem_wait_st();
                     fence_proxy_async_smem();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->afull);
+                    ok = combine_norms(nr2, ner2);
+                    if (!ok) break;
                 }
             }
             if (!ok) break;
             tc_fence_before();
-            if (valid && n_q != kQ) {
-                for (int l = 0; l < n_q; ++l) codes[frame * n_q + l] = (int16_t)win_codes[l];
-                ++done;
-            } else if (valid) {
-                uint4 pk;
-                pk.x = (uint32_t)(uint16_t)win_codes[0] | ((uint32_t)(uint16_t)win_codes[1] << 16);
-                pk.y = (uint32_t)(uint16_t)win_codes[2] | ((uint32_t)(uint16_t)win_codes[3] << 16);
-                pk.z = (uint32_t)(uint16_t)win_codes[4] | ((uint32_t)(uint16_t)win_codes[5] << 16);
-                pk.w = (uint32_t)(uint16_t)win_codes[6] | ((uint32_t)(uint16_t)win_codes[7] << 16);
-                *reinterpret_cast<uint4*>(codes + frame * kQ) = pk;
+            if (half == 0 && valid) {
+                if (n_q == kQ) {
+                    uint4 pk;
+                    pk.x = (uint32_t)(uint16_t)win_codes[0] | ((uint32_t)(uint16_t)win_codes[1] << 16);
+                    pk.y = (uint32_t)(uint16_t)win_codes[2] | ((uint32_t)(uint16_t)win_codes[3] << 16);
+                    pk.z = (uint32_t)(uint16_t)win_codes[4] | ((uint32_t)(uint16_t)win_codes[5] << 16);
+                    pk.w = (uint32_t)(uint16_t)win_codes[6] | ((uint32_t)(uint16_t)win_codes[7] << 16);
+                    *reinterpret_cast<uint4*>(codes + frame * kQ) = pk;
+                } else {
+                    for (int l = 0; l < n_q; ++l) codes[frame * n_q + l] = (int16_t)win_codes[l];
+                }
                 ++done;
             }
         }
