@@ -82,6 +82,10 @@ __device__ __forceinline__ float make_key(float s, int idx) {
 }
 __device__ __forceinline__ int key_index(float k) { return __float_as_int(k) & 0x7FF; }
 __device__ __forceinline__ float key_slack(float k) { return fabsf(k) * 4.8828125e-4f; }
+// Smallest raw score a key can stand for (an empty slot, +inf, stays +inf).
+__device__ __forceinline__ float key_lower(float k) {
+    return k < __int_as_float(0x7f800000) ? k - key_slack(k) : k;
+}
 
 struct Bars {
     uint64_t full[STAGES], empty[STAGES];
@@ -502,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float wthr = ts[0] + key_slack(ts[0]) + twoE;
                     int m = 0;
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) m += (ts[p] - key_slack(ts[p]) <= wthr) ? 1 : 0;
-                    const bool certified = ts[TOPK - 1] - key_slack(ts[TOPK - 1]) > wthr;
+                    for (int p = 0; p < TOPK; ++p) m += (key_lower(ts[p]) <= wthr) ? 1 : 0;
+                    const bool certified = key_lower(ts[TOPK - 1]) > wthr;
                     if (valid && !certified && !flagged) {
                         flagged = true;
                         const int slot = atomicAdd(rescan_count, 1);
