@@ -49,10 +49,11 @@ constexpr int A_CHUNK_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int RING_OFF = 0;
 constexpr int A_OFF = STAGES * STAGE_BYTES;             // 128 KiB
 constexpr int X_OFF = A_OFF + KCH * A_CHUNK_BYTES;      // 192 KiB: epilogue exchange area
-constexpr int XKEYS_OFF = X_OFF;                        // [BM][TOPK] float keys
-constexpr int XWIN_OFF = XKEYS_OFF + BM * 8 * 4;        // [BM] int winners
+constexpr int XKEYS_OFF = X_OFF;                        // [BM][TOPK + 2] keys, best, evicted
+constexpr int XWIN_OFF = XKEYS_OFF + BM * 10 * 4;       // [BM] int winners
 constexpr int XNORM_OFF = XWIN_OFF + BM * 4;            // [2][BM][2] partial norms
-constexpr int BAR_OFF = XNORM_OFF + 2 * BM * 2 * 4;
+constexpr int CN_OFF = XNORM_OFF + 2 * BM * 2 * 4;      // [2][K] ||c||^2 of the current / next level
+constexpr int BAR_OFF = CN_OFF + 2 * kK * 4;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;        // barriers, slack for 1 KiB alignment
 constexpr int TOPK = 8;
 constexpr int kEpiWarps = 8;            // two per TMEM lane quarter: column halves
@@ -97,21 +98,27 @@ struct Bars {
     int abort;
 };
 
-// Insert key k into the ascending list ts[0..7] (the largest falls off).
-__device__ __forceinline__ void insert_key(float (&ts)[TOPK], float k) {
+// Per-row candidate state for one level: a first-in-first-out list of keys
+// (slot 0 newest), the best key seen (always also pushed into the list), and
+// the smallest key the list has pushed out. Nothing outside the list can beat
+// best + 2E unless an evicted key could, which the evicted bound detects.
+struct Cands {
+    float ts[TOPK];
+    float best, evicted;
+};
+
+__device__ __forceinline__ void cands_reset(Cands& c) {
 #pragma unroll
-    for (int p = 0; p < TOPK; ++p) {
-        const float lo = fminf(ts[p], k);
-        k = fmaxf(ts[p], k);
-        ts[p] = lo;
-    }
+    for (int p = 0; p < TOPK; ++p) c.ts[p] = __int_as_float(0x7f800000);
+    c.best = c.evicted = __int_as_float(0x7f800000);
 }
 
-// Threshold above which a raw score can be dropped: it is outside the window
-// of the current best (and the best only improves), or it would fall off the
-// full list at once.
-__device__ __forceinline__ float scan_threshold(const float (&ts)[TOPK], float twoE) {
-    return fminf(ts[TOPK - 1] + key_slack(ts[TOPK - 1]), ts[0] + key_slack(ts[0]) + twoE);
+__device__ __forceinline__ void cands_push(Cands& c, float k) {
+    c.evicted = fminf(c.evicted, c.ts[TOPK - 1]);
+#pragma unroll
+    for (int p = TOPK - 1; p > 0; --p) c.ts[p] = c.ts[p - 1];
+    c.ts[0] = k;
+    c.best = fminf(c.best, k);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -287,6 +294,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        float* cn_s = reinterpret_cast<float*>(smem + CN_OFF);
+        const int etid = threadIdx.x - 64;  // 0..255 within the epilogue
+        // copy ||c||^2 of codebook l into shared buffer l & 1 (8 floats per thread)
+        auto stage_cn = [&](int l) {
+            const float4* src = reinterpret_cast<const float4*>(cnorm + (size_t)l * kK);
+            float4* dst = reinterpret_cast<float4*>(cn_s + (l & 1) * kK);
+            dst[etid] = __ldg(src + etid);
+            dst[etid + 256] = __ldg(src + etid + 256);
+        };
         float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
         int* xwin = reinterpret_cast<int*>(smem + XWIN_OFF);
         float* xnorm = reinterpret_cast<float*>(smem + XNORM_OFF);
@@ -417,13 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->afull);
+            stage_cn(0);  // visible after the barrier in combine_norms
             ok = combine_norms(nr2, ner2);
             if (!ok) break;
 
             int win_codes[kQ];
             bool flagged = false;
             for (int l = 0; l < n_q && ok; ++l) {
-                const float* cn = cnorm + (size_t)l * kK;
+                const float* cn = cn_s + (l & 1) * kK;
                 const float* book = C32 + (size_t)l * kK * kD;
                 const float4 cb = __ldg(reinterpret_cast<const float4*>(cbound) + l);
                 const float cmax = cb.x, cnmax = cb.y, ecmax = cb.z;
@@ -433,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float E = 2.f * dot_err * 1.0001f +
                                 kScoreRel * (cnmax + 2.f * (nr + ner) * (cmax + ecmax));
                 const float twoE = 2.f * E;
-                float ts[TOPK];
-#pragma unroll
-                for (int p = 0; p < TOPK; ++p) ts[p] = __int_as_float(0x7f800000);
+                Cands cs;
+                cands_reset(cs);
+                // raw scores above thr are outside the window of the best so far
                 float thr = __int_as_float(0x7f800000);
                 // ---- scan this half of the 16 score tiles of the codebook
                 for (int nt = 0; nt < NT; ++nt) {
@@ -444,34 +461,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++tcnt;
                     if (!ok) break;
                     tc_fence_after();
-#pragma unroll 1
+                    uint32_t v[2][32];
+                    tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64, v[0]);
+                    tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64 + 32, v[1]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
+#pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
-                        const int ch = half * 2 + c2;
-                        uint32_t v[32];
-                        tmem_ld32(trow + TMEM_SCORE + bsel * BN + ch * 32, v);
-                        tmem_wait_ld();
-                        if (c2 == 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
-                        }
-                        const int k0 = nt * BN + ch * 32;
+                        const int k0 = nt * BN + half * 64 + c2 * 32;
                         const float4* cn4 = reinterpret_cast<const float4*>(cn + k0);
                         float sc[32];
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 c = __ldg(cn4 + q4);
-                            sc[4 * q4 + 0] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 0]), c.x);
-                            sc[4 * q4 + 1] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 1]), c.y);
-                            sc[4 * q4 + 2] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 2]), c.z);
-                            sc[4 * q4 + 3] = fmaf(-2.f, __uint_as_float(v[4 * q4 + 3]), c.w);
+                            const float4 c = cn4[q4];
+                            sc[4 * q4 + 0] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 0]), c.x);
+                            sc[4 * q4 + 1] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 1]), c.y);
+                            sc[4 * q4 + 2] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 2]), c.z);
+                            sc[4 * q4 + 3] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w);
                         }
                         float g[8];
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4)
                             g[q4] = fminf(fmin3(sc[4 * q4], sc[4 * q4 + 1], sc[4 * q4 + 2]),
                                           sc[4 * q4 + 3]);
-                        const float cm = fminf(fmin3(g[0], g[1], g[2]), fmin3(g[3], g[4], fmin3(g[5], g[6], g[7])));
+                        const float cm = fminf(fmin3(g[0], g[1], g[2]),
+                                               fmin3(g[3], g[4], fmin3(g[5], g[6], g[7])));
                         // the chunk minimum tightens the window before its groups are scanned
                         thr = fminf(thr, cm + key_slack(cm) + twoE);
                         if (cm <= thr) {
@@ -481,39 +497,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                     for (int e = 0; e < 4; ++e) {
                                         const float sv = sc[4 * q4 + e];
-                                        if (sv <= thr) {
-                                            insert_key(ts, make_key(sv, k0 + 4 * q4 + e));
-                                            thr = scan_threshold(ts, twoE);
-                                        }
+                                        if (sv <= thr) cands_push(cs, make_key(sv, k0 + 4 * q4 + e));
                                     }
+                                    thr = fminf(thr, cs.best + key_slack(cs.best) + twoE);
                                 }
                             }
                         }
                     }
                 }
                 if (!ok) break;
+                if (l + 1 < n_q) stage_cn(l + 1);  // visible after the next barrier
                 // ---- merge the halves; certified window; float32 re-score
                 if (half == 1) {
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) xkeys[row * TOPK + p] = ts[p];
+                    for (int p = 0; p < TOPK; ++p) xkeys[row * 10 + p] = cs.ts[p];
+                    xkeys[row * 10 + 8] = cs.best;
+                    xkeys[row * 10 + 9] = cs.evicted;
                 }
                 ok = esync();
                 if (!ok) break;
                 int win = 0;
                 if (half == 0) {
+                    const float best = fminf(cs.best, xkeys[row * 10 + 8]);
+                    const float wthr = best + key_slack(best) + twoE;
+                    cs.evicted = fminf(cs.evicted, xkeys[row * 10 + 9]);
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) insert_key(ts, xkeys[row * TOPK + p]);
-                    const float wthr = ts[0] + key_slack(ts[0]) + twoE;
+                    for (int p = 0; p < TOPK; ++p) {
+                        const float k = xkeys[row * 10 + p];
+                        if (key_lower(k) <= wthr) cands_push(cs, k);
+                    }
                     int m = 0;
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) m += (key_lower(ts[p]) <= wthr) ? 1 : 0;
-                    const bool certified = key_lower(ts[TOPK - 1]) > wthr;
+                    for (int p = 0; p < TOPK; ++p) m += (key_lower(cs.ts[p]) <= wthr) ? 1 : 0;
+                    const bool certified = key_lower(cs.evicted) > wthr;
                     if (valid && !certified && !flagged) {
                         flagged = true;
                         const int slot = atomicAdd(rescan_count, 1);
                         if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
                     }
-                    win = key_index(ts[0]);
+                    win = key_index(best);
                     if (__any_sync(0xffffffffu, m > 1)) {
                         float dot[TOPK];
 #pragma unroll
@@ -524,9 +546,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_wait_ld();
 #pragma unroll
                             for (int p = 0; p < TOPK; ++p) {
-                                if (p < m) {
+                                if (m > 1 && key_lower(cs.ts[p]) <= wthr) {
                                     const float4* c4 = reinterpret_cast<const float4*>(
-                                        book + (size_t)key_index(ts[p]) * kD + ch * 32);
+                                        book + (size_t)key_index(cs.ts[p]) * kD + ch * 32);
                                     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                                     for (int q4 = 0; q4 < 8; ++q4) {
@@ -540,17 +562,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                         }
-                        float best = __int_as_float(0x7f800000);
+                        if (m > 1) {
+                            float bs = __int_as_float(0x7f800000);
+                            win = 0x7fffffff;
 #pragma unroll
-                        for (int p = 0; p < TOPK; ++p) {
-                            if (p < m) {
-                                const int k = key_index(ts[p]);
-                                const float e = fmaf(-2.f, dot[p], __ldg(cn + k));
-                                if (e < best || (e == best && k < win)) {
-                                    best = e;
-                                    win = k;
+                            for (int p = 0; p < TOPK; ++p) {
+                                if (key_lower(cs.ts[p]) <= wthr) {
+                                    const int k = key_index(cs.ts[p]);
+                                    const float e = fmaf(-2.f, dot[p], __ldg(cnorm + (size_t)l * kK + k));
+                                    if (e < bs || (e == bs && k < win)) {
+                                        bs = e;
+                                        win = k;
+                                    }
                                 }
                             }
+                            if (win >= kK) win = key_index(best);
                         }
                     }
                     win_codes[l] = win;
