@@ -325,6 +325,10 @@ def run_ours(args, rank, world, local_rank):
     roofline["kernel"] = dominant["kernel"]
     roofline["peak_source"] = (f"{peaks['source']} "
                                f"{'bf16_tflops_sustained' if dominant['bound'] == 'tensor' else 'hbm_gbs'}")
+    if args.self_profile and do_enc:
+        _, cyc = q.encode_profile(z, out=codes, stream=stream)
+        total = max(cyc["cta_total"], 1)
+        kernels[0]["self_profile_share"] = {k: round(v / total, 4) for k, v in cyc.items()}
     launches_per_step = (2 if do_enc else 0) + (1 if do_dec else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,
@@ -437,6 +441,8 @@ def main():
     ap.add_argument("--calls", type=int, default=1000, help="streaming workload: calls per B")
     ap.add_argument("--frames", type=int, default=None,
                     help="shrink the workload (for profiler captures); default: full size")
+    ap.add_argument("--self-profile", action="store_true",
+                    help="add the encode kernel's per-role cycle shares (one extra untimed call)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

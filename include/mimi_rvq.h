@@ -118,6 +118,22 @@ int mimi_rvq_encode_ex(mimi_rvq_t h, const void *latents, int dtype, int64_t N, 
                        int variant, int16_t *codes, struct CUstream_st *stream);
 
 /*
+ * Diagnostic: mimi_rvq_encode (n_q = 8, variant 0, N <= 1 048 576) that also
+ * adds, into cycles[0..15] (device, caller-zeroed, uint64), the SM clock
+ * cycles each role of the tensor-core kernel spent, summed over CTAs:
+ *   0 TMA producer waiting for a free stage      1 MMA waiting for operand tiles
+ *   2 MMA waiting for a drained score buffer     3 MMA waiting for a level's A operand
+ *   4 MMA waiting for staged latents             5 epilogue waiting for a score tile
+ *   6 epilogue scanning scores                   7 epilogue merge / window / re-score
+ *   8 epilogue residual update                   9 epilogue latent staging, y read-out
+ *  10 epilogue barrier waits                    11 whole CTA
+ * (counters 5..10 are one epilogue thread per CTA). Codes are the same as
+ * mimi_rvq_encode's.
+ */
+int mimi_rvq_encode_profile(mimi_rvq_t h, const void *latents, int dtype, int64_t N,
+                            int16_t *codes, uint64_t *cycles, struct CUstream_st *stream);
+
+/*
  * The projection step alone: latents [N][512] -> y = W_in . z [N][256] fp32,
  * computed exactly as encode computes it (split-precision bf16 products on
  * the tensor cores, float32 accumulation).

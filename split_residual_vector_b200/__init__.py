@@ -21,7 +21,8 @@ STATUS = {0: "ok", -1: "invalid argument", -2: "out of device memory", -3: "CUDA
 LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmimi_rvq.so")
 EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_encode_ex",
            "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
-           "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror")
+           "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror",
+           "mimi_rvq_encode_profile")
 
 _lib = None
 
@@ -51,6 +52,8 @@ def library() -> ctypes.CDLL:
     for name in ("mimi_rvq_encode_ex", "mimi_rvq_encode_scan"):
         getattr(lib, name).argtypes = [vp, vp, ci, i64, ci, ci, vp, vp]
         getattr(lib, name).restype = ci
+    lib.mimi_rvq_encode_profile.argtypes = [vp, vp, ci, i64, vp, vp, vp]
+    lib.mimi_rvq_encode_profile.restype = ci
     lib.mimi_rvq_project.argtypes = [vp, vp, ci, i64, vp, vp]
     lib.mimi_rvq_project.restype = ci
     lib.mimi_rvq_decode_ex.argtypes = [vp, vp, i64, ci, vp, vp]
@@ -191,6 +194,24 @@ class Quantizer:
                                               _stream(stream))
         _check(st, "mimi_rvq_decode")
         return out
+
+    PROFILE_SLOTS = ("producer_wait_stage", "mma_wait_operands", "mma_wait_score_buffer",
+                     "mma_wait_level_operand", "mma_wait_latents", "epi_wait_score_tile",
+                     "epi_scan", "epi_pick", "epi_update", "epi_stage", "epi_barrier",
+                     "cta_total")
+
+    def encode_profile(self, latents, out=None, stream=None):
+        """Encode and return (codes, {role: cycles summed over CTAs}) from the kernel's
+        self-profile."""
+        import torch
+        n, dt = self._latents(latents)
+        out = self._codes_out(n, out)
+        cyc = torch.zeros(16, dtype=torch.int64, device=self.device)
+        _check(library().mimi_rvq_encode_profile(self._h, latents.data_ptr(), dt, n,
+                                                 out.data_ptr(), cyc.data_ptr(), _stream(stream)),
+               "mimi_rvq_encode_profile")
+        vals = cyc.cpu().tolist()
+        return out, dict(zip(self.PROFILE_SLOTS, vals))
 
     def get_error(self, stream=None) -> int:
         """Synchronise the stream; return and clear the device error status (0 = ok)."""

@@ -217,6 +217,21 @@ int mimi_rvq_encode_step(mimi_rvq_t h, const void* frames, int dtype, int B, int
     return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, kQ, 0, codes, stream);
 }
 
+int mimi_rvq_encode_profile(mimi_rvq_t h, const void* latents, int dtype, int64_t N,
+                            int16_t* codes, uint64_t* cycles, struct CUstream_st* stream) {
+    if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
+    if (N > mimi::kRescanCapacity) return MIMI_RVQ_EINVAL;
+    const int c = check_common(h, latents, codes, N);
+    if (c <= 0) return c;
+    if (!device_pointer(cycles)) return MIMI_RVQ_EINVAL;
+    cudaError_t e = cudaMemsetAsync(h->t.rescan_count, 0, sizeof(int), stream);
+    if (e == cudaSuccess)
+        e = mimi::launch_encode_tc(h->t, latents, dtype, N, kQ, 0, codes, nullptr, stream,
+                                   h->num_sms, reinterpret_cast<unsigned long long*>(cycles));
+    if (e == cudaSuccess) e = mimi::launch_rescan(h->t, latents, dtype, kQ, 0, codes, stream);
+    return from_cuda(e);
+}
+
 int mimi_rvq_project(mimi_rvq_t h, const void* latents, int dtype, int64_t N, float* y,
                      struct CUstream_st* stream) {
     if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;

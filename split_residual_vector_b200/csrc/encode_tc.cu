@@ -88,6 +88,24 @@ __device__ __forceinline__ float key_lower(float k) {
     return k < __int_as_float(0x7f800000) ? k - key_slack(k) : k;
 }
 
+// Optional self-profile: cycles each role spends waiting or working, summed
+// over CTAs into prof[kProfSlots] (diagnostic entry point only).
+enum ProfSlot {
+    P_PROD_EMPTY = 0,   // producer waiting for a free ring stage
+    P_MMA_FULL,         // MMA waiting for codebook / weight tiles
+    P_MMA_TEMPTY,       // MMA waiting for a drained TMEM score buffer
+    P_MMA_AFULL,        // MMA waiting for the next level's A operand
+    P_MMA_ZFULL,        // MMA waiting for staged latents
+    P_EPI_TFULL,        // epilogue (one thread) waiting for a score tile
+    P_EPI_SCAN,         // epilogue scanning score tiles
+    P_EPI_PICK,         // epilogue merge, window, re-score
+    P_EPI_UPDATE,       // epilogue residual update (including its waits)
+    P_EPI_STAGE,        // epilogue latent staging and y read-out
+    P_EPI_ESYNC,        // epilogue barrier waits
+    P_CTA_TOTAL,        // whole CTA
+    kProfSlots = 16
+};
+
 struct Bars {
     uint64_t full[STAGES], empty[STAGES];
     uint64_t zfull[2], zempty[2];
@@ -127,7 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* __restrict__ cnorm, const float* __restrict__ cbound,
                 const void* __restrict__ z, int dtype, int64_t n, int n_q, int variant,
                 int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
-                int* rescan_count, int* rescan_list, unsigned long long* stats) {
+                int* rescan_count, int* rescan_list, unsigned long long* stats,
+                unsigned long long* prof) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -176,16 +195,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    const long long t_cta0 = clock64();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
+            long long p_empty = 0;
             auto load = [&](const CUtensorMap* tm, int x, int y) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&bars->empty[s], ph ^ 1, abort, err)) return false;
+                const long long t0 = clock64();
+                const bool r = mbar_wait(&bars->empty[s], ph ^ 1, abort, err);
+                p_empty += clock64() - t0;
+                if (!r) return false;
                 mbar_arrive_expect_tx(&bars->full[s], STAGE_BYTES);
                 tma_load_2d(smem + RING_OFF + s * STAGE_BYTES, tm, &bars->full[s], x, y);
                 ++it;
@@ -205,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t first = it > STAGES ? it - STAGES : 0;
             for (uint32_t j = first; j < it; ++j)
                 mbar_wait(&bars->full[j % STAGES], (j / STAGES) & 1, abort, err);
+            if (prof) atomicAdd(prof + P_PROD_EMPTY, (unsigned long long)p_empty);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -212,11 +237,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc = idesc_bf16_f32(BM, BN);
             uint32_t it = 0, zuse[2] = {0, 0}, acnt = 0, tcnt = 0;
             bool ok = true;
+            long long p_full = 0, p_tempty = 0, p_afull = 0, p_zfull = 0;
+            auto twait = [&](uint64_t* bar, uint32_t parity, long long& acc) {
+                const long long t0 = clock64();
+                const bool r = mbar_wait(bar, parity, abort, err);
+                acc += clock64() - t0;
+                return r;
+            };
             for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
                 // projection: y = z_hi W_hi + z_lo W_hi + z_hi W_lo into columns [0, 256)
                 for (int kc = 0; kc < PKCH && ok; ++kc) {
                     const int zb = kc & 1;
-                    ok = mbar_wait(&bars->zfull[zb], zuse[zb] & 1, abort, err);
+                    ok = twait(&bars->zfull[zb], zuse[zb] & 1, p_zfull);
                     ++zuse[zb];
                     if (!ok) break;
                     tc_fence_after();
@@ -224,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a_lo = a_hi + A_CHUNK_BYTES;
                     for (int g = 0; g < 4 && ok; ++g) {
                         const int s = it % STAGES;
-                        ok = mbar_wait(&bars->full[s], (it / STAGES) & 1, abort, err);
+                        ok = twait(&bars->full[s], (it / STAGES) & 1, p_full);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t b = ring + s * STAGE_BYTES;
@@ -248,20 +280,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the eight codebooks
                 for (int l = 0; l < n_q && ok; ++l) {
                     if (l == 0 || updates_after(l - 1)) {
-                        ok = mbar_wait(&bars->afull, acnt & 1, abort, err);
+                        ok = twait(&bars->afull, acnt & 1, p_afull);
                         ++acnt;
                         if (!ok) break;
                         tc_fence_after();
                     }
                     for (int nt = 0; nt < NT && ok; ++nt) {
                         const int bsel = tcnt & 1;
-                        ok = mbar_wait(&bars->tempty[bsel], ((tcnt >> 1) & 1) ^ 1, abort, err);
+                        ok = twait(&bars->tempty[bsel], ((tcnt >> 1) & 1) ^ 1, p_tempty);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t d = tmem + TMEM_SCORE + bsel * BN;
                         for (int kc = 0; kc < KCH && ok; ++kc) {
                             const int s = it % STAGES;
-                            ok = mbar_wait(&bars->full[s], (it / STAGES) & 1, abort, err);
+                            ok = twait(&bars->full[s], (it / STAGES) & 1, p_full);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t b = ring + s * STAGE_BYTES;
@@ -282,6 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // drain: every issued MMA must complete before TMEM is freed
             umma_commit(&bars->drain);
             mbar_wait(&bars->drain, 0, abort, err);
+            if (prof) {
+                atomicAdd(prof + P_MMA_FULL, (unsigned long long)p_full);
+                atomicAdd(prof + P_MMA_TEMPTY, (unsigned long long)p_tempty);
+                atomicAdd(prof + P_MMA_AFULL, (unsigned long long)p_afull);
+                atomicAdd(prof + P_MMA_ZFULL, (unsigned long long)p_zfull);
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -309,6 +347,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t zuse[2] = {0, 0}, aecnt = 0, tcnt = 0, tile_iter = 0;
         bool ok = true;
         unsigned long long done = 0;
+        long long p_tfull = 0, p_scan = 0, p_pick = 0, p_update = 0, p_stage = 0, p_esync = 0;
+        long long t_mark = clock64();
+        // attribute the cycles since the last mark to one counter
+        auto mark = [&](long long& acc) {
+            const long long t = clock64();
+            acc += t - t_mark;
+            t_mark = t;
+        };
         // every lane of the warp takes the same branch after a wait, so the
         // .sync.aligned TMEM loads below are never reached divergently
         auto ewait = [&](uint64_t* bar, uint32_t parity) {
@@ -340,7 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ephase = 0;
         auto esync = [&]() {
             mbar_arrive(&bars->ebar);
+            const long long t0 = clock64();
             const bool r = mbar_wait(&bars->ebar, ephase & 1, abort, err);
+            p_esync += clock64() - t0;
             ++ephase;
             return __all_sync(0xffffffffu, r) != 0;
         };
@@ -437,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = combine_norms(nr2, ner2);
             if (!ok) break;
 
+            mark(p_stage);
             int win_codes[kQ];
             bool flagged = false;
             for (int l = 0; l < n_q && ok; ++l) {
@@ -457,7 +506,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- scan this half of the 16 score tiles of the codebook
                 for (int nt = 0; nt < NT; ++nt) {
                     const int bsel = tcnt & 1;
+                    mark(p_scan);
                     ok = ewait(&bars->tfull[bsel], (tcnt >> 1) & 1);
+                    mark(p_tfull);
                     ++tcnt;
                     if (!ok) break;
                     tc_fence_after();
@@ -506,6 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (!ok) break;
+                mark(p_scan);
                 if (l + 1 < n_q) stage_cn(l + 1);  // visible after the next barrier
                 // ---- merge the halves; certified window; float32 re-score
                 if (half == 1) {
@@ -582,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     win_codes[l] = win;
                     xwin[row] = win;
                 }
+                mark(p_pick);
                 // ---- residual update r -= c_win for the next level, split by halves
                 if (updates_after(l)) {
                     ok = esync();
@@ -618,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) mbar_arrive(&bars->afull);
                     ok = combine_norms(nr2, ner2);
                     if (!ok) break;
+                    mark(p_update);
                 }
             }
             if (!ok) break;
@@ -636,6 +690,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++done;
             }
         }
+        mark(p_stage);
+        if (prof && warp == 2 && lane == 0) {
+            atomicAdd(prof + P_EPI_TFULL, (unsigned long long)p_tfull);
+            atomicAdd(prof + P_EPI_SCAN, (unsigned long long)p_scan);
+            atomicAdd(prof + P_EPI_PICK, (unsigned long long)p_pick);
+            atomicAdd(prof + P_EPI_UPDATE, (unsigned long long)p_update);
+            atomicAdd(prof + P_EPI_STAGE, (unsigned long long)p_stage);
+            atomicAdd(prof + P_EPI_ESYNC, (unsigned long long)p_esync);
+        }
         // count frames (one atomic per warp)
         for (int o = 16; o > 0; o >>= 1) done += __shfl_xor_sync(0xffffffffu, done, o);
         if (lane == 0 && done) atomicAdd(&stats[0], done);
@@ -644,6 +707,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+    if (prof && threadIdx.x == 0)
+        atomicAdd(prof + P_CTA_TOTAL, (unsigned long long)(clock64() - t_cta0));
 }
 
 }  // namespace
@@ -655,14 +720,14 @@ cudaError_t encode_tc_configure() {
 
 cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                              int variant, int16_t* codes, float* y_out, cudaStream_t s,
-                             int max_ctas) {
+                             int max_ctas, unsigned long long* prof) {
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + BM - 1) / BM;
     const int grid = (int)(tiles < max_ctas ? tiles : max_ctas);
     k_encode_tc<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm,
                                                    t.cbound, z, dtype, n, n_q, variant, codes,
                                                    y_out, t.err, t.rescan_count, t.rescan_list,
-                                                   t.stats);
+                                                   t.stats, prof);
     return cudaGetLastError();
 }
 

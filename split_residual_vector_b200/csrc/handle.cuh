@@ -48,9 +48,10 @@ cudaError_t prep_tables(Tables& t, const float* W_out, cudaStream_t s);
 cudaError_t encode_tc_configure();  // once per device, before the first launch
 // n_q codebooks (0 = projection only, writing y_out [n][256]); codes [n][n_q];
 // variant 1 runs the acoustic RVQ on y - S_s.
+// prof (nullable, device, 16 counters): per-role cycle counters, see ProfSlot.
 cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                              int variant, int16_t* codes, float* y_out, cudaStream_t s,
-                             int max_ctas);
+                             int max_ctas, unsigned long long* prof = nullptr);
 // encode_scan.cu
 cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                                int variant, int16_t* codes, cudaStream_t s);
