@@ -178,6 +178,28 @@ int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st *stream);
 int mimi_rvq_stats(mimi_rvq_t h, struct CUstream_st *stream, int64_t *frames_encoded,
                    int64_t *frames_rescanned);
 
+/*
+ * Encode without a handle and without allocating device memory, for callers
+ * that cannot call cudaMalloc: a host that lets libraries use only the device
+ * buffers it hands them, or a real-time audio thread, where cudaMalloc and
+ * cudaFree may synchronise the device. The pages have no counterpart to this
+ * call; it is part of this library's interface, not of the method.
+ *   codebooks [8][2048][256] fp32 (only the first n_q are read), W_in
+ *   [256][512] fp32, latents [N][512] (MIMI_RVQ_F32 or MIMI_RVQ_BF16),
+ *   codes [N][n_q] int16 out; all device pointers owned by the caller.
+ * Same arithmetic and codes as mimi_rvq_encode_scan (the float32 full scan:
+ * exact float32 scores, slow). Its one piece of scratch, the squared codeword
+ * norms, lives in a 64 KiB static device array (at most 8 codebooks of 2048;
+ * n_q outside 1..8 returns MIMI_RVQ_EINVAL) that every GPU loading the
+ * library holds until exit. The first call on a device looks up that array's
+ * address; make it before any stream capture. Every call shares the array and
+ * rewrites it, so calls that overlap on the GPU (other streams, other host
+ * threads) race: serialise them.
+ */
+int mimi_rvq_encode_noalloc(const float *codebooks, const float *W_in, const void *latents,
+                            int dtype, int64_t N, int n_q, int16_t *codes,
+                            struct CUstream_st *stream);
+
 /* Static English text for a status code. */
 const char *mimi_rvq_strerror(int status);
 
