@@ -44,18 +44,18 @@ constexpr int NT = kK / BN;             // 16 score tiles per codebook
 constexpr int KCH = kD / BK;            // 4 K chunks per score tile
 constexpr int PKCH = kDin / BK;         // 8 K chunks of the projection
 constexpr int STAGES = 8;
+constexpr int TOPK = 8;                 // candidate list length per row and half
 constexpr int STAGE_BYTES = BN * BK * 2;        // 16 KiB
 constexpr int A_CHUNK_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int RING_OFF = 0;
 constexpr int A_OFF = STAGES * STAGE_BYTES;             // 128 KiB
 constexpr int X_OFF = A_OFF + KCH * A_CHUNK_BYTES;      // 192 KiB: epilogue exchange area
-constexpr int XKEYS_OFF = X_OFF;                        // [BM][TOPK + 2] keys, best, evicted
-constexpr int XWIN_OFF = XKEYS_OFF + BM * 10 * 4;       // [BM] int winners
-constexpr int XNORM_OFF = XWIN_OFF + BM * 4;            // [2][BM][2] partial norms
-constexpr int CN_OFF = XNORM_OFF + 2 * BM * 2 * 4;      // [2][K] ||c||^2 of the current / next level
-constexpr int BAR_OFF = CN_OFF + 2 * kK * 4;
+constexpr int XKEYS_OFF = X_OFF;                        // [2][BM][TOPK + 2] keys, best, evicted
+constexpr int XDOT_OFF = XKEYS_OFF + 2 * BM * 10 * 4;   // [2][BM][TOPK] partial re-score dots
+constexpr int XNORM_OFF = XDOT_OFF + 2 * BM * TOPK * 4; // [2][BM][2] partial norms
+constexpr int CN_OFF = XNORM_OFF + 2 * BM * 2 * 4;      // [K] ||c||^2 of the level being scanned
+constexpr int BAR_OFF = CN_OFF + kK * 4;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;        // barriers, slack for 1 KiB alignment
-constexpr int TOPK = 8;
 constexpr int kEpiWarps = 8;            // two per TMEM lane quarter: column halves
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t TMEM_COLS = 512;
@@ -334,15 +334,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         float* cn_s = reinterpret_cast<float*>(smem + CN_OFF);
         const int etid = threadIdx.x - 64;  // 0..255 within the epilogue
-        // copy ||c||^2 of codebook l into shared buffer l & 1 (8 floats per thread)
+        // copy ||c||^2 of codebook l into shared memory (8 floats per thread); callers
+        // place it after a barrier that ends all reads of the previous level's copy
+        // and before one that precedes the next scan
         auto stage_cn = [&](int l) {
             const float4* src = reinterpret_cast<const float4*>(cnorm + (size_t)l * kK);
-            float4* dst = reinterpret_cast<float4*>(cn_s + (l & 1) * kK);
+            float4* dst = reinterpret_cast<float4*>(cn_s);
             dst[etid] = __ldg(src + etid);
             dst[etid + 256] = __ldg(src + etid + 256);
         };
         float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
-        int* xwin = reinterpret_cast<int*>(smem + XWIN_OFF);
+        float* xdot = reinterpret_cast<float*>(smem + XDOT_OFF);
         float* xnorm = reinterpret_cast<float*>(smem + XNORM_OFF);
         uint32_t zuse[2] = {0, 0}, aecnt = 0, tcnt = 0, tile_iter = 0;
         bool ok = true;
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int win_codes[kQ];
             bool flagged = false;
             for (int l = 0; l < n_q && ok; ++l) {
-                const float* cn = cn_s + (l & 1) * kK;
+                const float* cn = cn_s;
                 const float* book = C32 + (size_t)l * kK * kD;
                 const float4 cb = __ldg(reinterpret_cast<const float4*>(cbound) + l);
                 const float cmax = cb.x, cnmax = cb.y, ecmax = cb.z;
@@ -558,120 +560,144 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 mark(p_scan);
-                if (l + 1 < n_q) stage_cn(l + 1);  // visible after the next barrier
-                // ---- merge the halves; certified window; float32 re-score
-                if (half == 1) {
+                // ---- exchange both halves' lists; both merge them the same way
+                {
+                    float* mine = xkeys + (half * BM + row) * 10;
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) xkeys[row * 10 + p] = cs.ts[p];
-                    xkeys[row * 10 + 8] = cs.best;
-                    xkeys[row * 10 + 9] = cs.evicted;
+                    for (int p = 0; p < TOPK; ++p) mine[p] = cs.ts[p];
+                    mine[8] = cs.best;
+                    mine[9] = cs.evicted;
                 }
                 ok = esync();
                 if (!ok) break;
-                int win = 0;
-                if (half == 0) {
-                    const float best = fminf(cs.best, xkeys[row * 10 + 8]);
-                    const float wthr = best + key_slack(best) + twoE;
-                    cs.evicted = fminf(cs.evicted, xkeys[row * 10 + 9]);
+                if (l + 1 < n_q) stage_cn(l + 1);  // every read of this level's copy is done
+                {
+                    const float* k0 = xkeys + row * 10;
+                    const float* k1 = xkeys + (BM + row) * 10;
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) cs.ts[p] = k0[p];
+                    cs.best = k0[8];
+                    cs.evicted = k0[9];
+                    const float best1 = k1[8];
+                    const float wthr0 = fminf(cs.best, best1);
+                    const float wthr = wthr0 + key_slack(wthr0) + twoE;
+                    cs.evicted = fminf(cs.evicted, k1[9]);
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) {
-                        const float k = xkeys[row * 10 + p];
+                        const float k = k1[p];
                         if (key_lower(k) <= wthr) cands_push(cs, k);
                     }
+                    cs.best = fminf(cs.best, best1);
                     int m = 0;
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) m += (key_lower(cs.ts[p]) <= wthr) ? 1 : 0;
                     const bool certified = key_lower(cs.evicted) > wthr;
-                    if (valid && !certified && !flagged) {
+                    if (half == 0 && valid && !certified && !flagged) {
                         flagged = true;
                         const int slot = atomicAdd(rescan_count, 1);
                         if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
                     }
-                    win = key_index(best);
-                    if (__any_sync(0xffffffffu, m > 1)) {
-                        float dot[TOPK];
+                    // ---- float32 re-score of the window: each half dots its own 128
+                    //      dimensions of r with every candidate, 64 at a time
+                    float dot[TOPK];
 #pragma unroll
-                        for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
-                        for (int ch = 0; ch < kD / 32; ++ch) {
-                            uint32_t v[32];
-                            tmem_ld32(trow + ch * 32, v);
+                    for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
+                    if (__any_sync(0xffffffffu, m > 1)) {
+#pragma unroll 1
+                        for (int b = 0; b < 2; ++b) {
+                            uint32_t v[2][32];
+                            tmem_ld32(trow + (half * 4 + 2 * b) * 32, v[0]);
+                            tmem_ld32(trow + (half * 4 + 2 * b + 1) * 32, v[1]);
                             tmem_wait_ld();
 #pragma unroll
                             for (int p = 0; p < TOPK; ++p) {
                                 if (m > 1 && key_lower(cs.ts[p]) <= wthr) {
                                     const float4* c4 = reinterpret_cast<const float4*>(
-                                        book + (size_t)key_index(cs.ts[p]) * kD + ch * 32);
+                                        book + (size_t)key_index(cs.ts[p]) * kD + half * 128 + b * 64);
+                                    float4 c[16];
+#pragma unroll
+                                    for (int q4 = 0; q4 < 16; ++q4) c[q4] = __ldg(c4 + q4);
                                     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                                    for (int q4 = 0; q4 < 8; ++q4) {
-                                        const float4 c = __ldg(c4 + q4);
-                                        a0 = fmaf(__uint_as_float(v[4 * q4 + 0]), c.x, a0);
-                                        a1 = fmaf(__uint_as_float(v[4 * q4 + 1]), c.y, a1);
-                                        a0 = fmaf(__uint_as_float(v[4 * q4 + 2]), c.z, a0);
-                                        a1 = fmaf(__uint_as_float(v[4 * q4 + 3]), c.w, a1);
+                                    for (int q4 = 0; q4 < 16; ++q4) {
+                                        const uint32_t* vv = v[q4 >> 3] + 4 * (q4 & 7);
+                                        a0 = fmaf(__uint_as_float(vv[0]), c[q4].x, a0);
+                                        a1 = fmaf(__uint_as_float(vv[1]), c[q4].y, a1);
+                                        a0 = fmaf(__uint_as_float(vv[2]), c[q4].z, a0);
+                                        a1 = fmaf(__uint_as_float(vv[3]), c[q4].w, a1);
                                     }
                                     dot[p] += a0 + a1;
                                 }
                             }
                         }
-                        if (m > 1) {
-                            float bs = __int_as_float(0x7f800000);
-                            win = 0x7fffffff;
-#pragma unroll
-                            for (int p = 0; p < TOPK; ++p) {
-                                if (key_lower(cs.ts[p]) <= wthr) {
-                                    const int k = key_index(cs.ts[p]);
-                                    const float e = fmaf(-2.f, dot[p], __ldg(cnorm + (size_t)l * kK + k));
-                                    if (e < bs || (e == bs && k < win)) {
-                                        bs = e;
-                                        win = k;
-                                    }
-                                }
-                            }
-                            if (win >= kK) win = key_index(best);
-                        }
                     }
-                    win_codes[l] = win;
-                    xwin[row] = win;
-                }
-                mark(p_pick);
-                // ---- residual update r -= c_win for the next level, split by halves
-                if (updates_after(l)) {
+                    float* xd = xdot + (half * BM + row) * TOPK;
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) xd[p] = dot[p];
                     ok = esync();
                     if (!ok) break;
-                    win = xwin[row];
-                    ok = ewait(&bars->aempty, aecnt & 1);
-                    ++aecnt;
-                    if (!ok) break;
-                    nr2 = 0.f;
-                    ner2 = 0.f;
-                    const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD);
-                    for (int c4i = 0; c4i < 4; ++c4i) {
-                        const int ch = half * 4 + c4i;
-                        uint32_t v[32];
-                        tmem_ld32(trow + ch * 32, v);
-                        float4 c[8];
+                    int win = key_index(cs.best);
+                    if (m > 1) {
+                        const float* d0 = xdot + row * TOPK;
+                        const float* d1 = xdot + (BM + row) * TOPK;
+                        float bs = __int_as_float(0x7f800000);
+                        int bw = 0x7fffffff;
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) c[q4] = __ldg(c4 + ch * 8 + q4);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            v[4 * q4 + 0] = __float_as_uint(__uint_as_float(v[4 * q4 + 0]) - c[q4].x);
-                            v[4 * q4 + 1] = __float_as_uint(__uint_as_float(v[4 * q4 + 1]) - c[q4].y);
-                            v[4 * q4 + 2] = __float_as_uint(__uint_as_float(v[4 * q4 + 2]) - c[q4].z);
-                            v[4 * q4 + 3] = __float_as_uint(__uint_as_float(v[4 * q4 + 3]) - c[q4].w);
+                        for (int p = 0; p < TOPK; ++p) {
+                            if (key_lower(cs.ts[p]) <= wthr) {
+                                const int k = key_index(cs.ts[p]);
+                                const float e = fmaf(-2.f, d0[p] + d1[p], __ldg(cnorm + (size_t)l * kK + k));
+                                if (e < bs || (e == bs && k < bw)) {
+                                    bs = e;
+                                    bw = k;
+                                }
+                            }
                         }
-                        tmem_st32(trow + ch * 32, v);
-                        write_a_chunk(ch, v, nr2, ner2);
+                        if (bw < kK) win = bw;
                     }
-                    tmem_wait_st();
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->afull);
-                    ok = combine_norms(nr2, ner2);
-                    if (!ok) break;
-                    mark(p_update);
+                    win_codes[l] = win;
+                    mark(p_pick);
+                    // ---- residual update r -= c_win for the next level, split by halves
+                    if (updates_after(l)) {
+                        ok = ewait(&bars->aempty, aecnt & 1);
+                        ++aecnt;
+                        if (!ok) break;
+                        nr2 = 0.f;
+                        ner2 = 0.f;
+                        const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD + half * 128);
+#pragma unroll 1
+                        for (int b = 0; b < 2; ++b) {
+                            uint32_t v[2][32];
+                            tmem_ld32(trow + (half * 4 + 2 * b) * 32, v[0]);
+                            tmem_ld32(trow + (half * 4 + 2 * b + 1) * 32, v[1]);
+                            float4 c[16];
+#pragma unroll
+                            for (int q4 = 0; q4 < 16; ++q4) c[q4] = __ldg(c4 + b * 16 + q4);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+                                for (int q4 = 0; q4 < 8; ++q4) {
+                                    const float4 cc = c[h2 * 8 + q4];
+                                    v[h2][4 * q4 + 0] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 0]) - cc.x);
+                                    v[h2][4 * q4 + 1] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 1]) - cc.y);
+                                    v[h2][4 * q4 + 2] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 2]) - cc.z);
+                                    v[h2][4 * q4 + 3] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 3]) - cc.w);
+                                }
+                                const int ch = half * 4 + 2 * b + h2;
+                                tmem_st32(trow + ch * 32, v[h2]);
+                                write_a_chunk(ch, v[h2], nr2, ner2);
+                            }
+                        }
+                        tmem_wait_st();
+                        fence_proxy_async_smem();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->afull);
+                        ok = combine_norms(nr2, ner2);
+                        if (!ok) break;
+                        mark(p_update);
+                    }
                 }
             }
             if (!ok) break;
