@@ -198,7 +198,7 @@ class Quantizer:
     PROFILE_SLOTS = ("producer_wait_stage", "mma_wait_operands", "mma_wait_score_buffer",
                      "mma_wait_level_operand", "mma_wait_latents", "epi_wait_score_tile",
                      "epi_scan", "epi_pick", "epi_update", "epi_stage", "epi_barrier",
-                     "cta_total")
+                     "cta_total", "scan_tmem", "scan_math", "scan_push")
 
     def encode_profile(self, latents, out=None, stream=None):
         """Encode and return (codes, {role: cycles summed over CTAs}) from the kernel's

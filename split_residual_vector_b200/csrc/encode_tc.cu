@@ -103,6 +103,9 @@ enum ProfSlot {
     P_EPI_STAGE,        // epilogue latent staging and y read-out
     P_EPI_ESYNC,        // epilogue barrier waits
     P_CTA_TOTAL,        // whole CTA
+    P_SCAN_TMEM,        // part of P_EPI_SCAN: TMEM loads of score tiles
+    P_SCAN_MATH,        // part of P_EPI_SCAN: scores, group and chunk minima
+    P_SCAN_PUSH,        // part of P_EPI_SCAN: window checks and list pushes
     kProfSlots = 16
 };
 
@@ -116,10 +119,10 @@ struct Bars {
     int abort;
 };
 
-// Per-row candidate state for one level: a first-in-first-out list of keys
-// (slot 0 newest), the best key seen (always also pushed into the list), and
-// the smallest key the list has pushed out. Nothing outside the list can beat
-// best + 2E unless an evicted key could, which the evicted bound detects.
+// Per-row candidate state for one level: the best key seen, an ascending list
+// of the best other keys that were inside the window when they appeared, and
+// the smallest key that has fallen off the end of the list. Inserting +inf is
+// a no-op, so callers insert unconditionally (no divergent branches).
 struct Cands {
     float ts[TOPK];
     float best, evicted;
@@ -131,12 +134,45 @@ __device__ __forceinline__ void cands_reset(Cands& c) {
     c.best = c.evicted = __int_as_float(0x7f800000);
 }
 
-__device__ __forceinline__ void cands_push(Cands& c, float k) {
-    c.evicted = fminf(c.evicted, c.ts[TOPK - 1]);
+__device__ __forceinline__ void cands_insert(Cands& c, float k) {
 #pragma unroll
-    for (int p = TOPK - 1; p > 0; --p) c.ts[p] = c.ts[p - 1];
-    c.ts[0] = k;
-    c.best = fminf(c.best, k);
+    for (int p = 0; p < TOPK; ++p) {
+        const float lo = fminf(c.ts[p], k);
+        k = fmaxf(c.ts[p], k);
+        c.ts[p] = lo;
+    }
+    c.evicted = fminf(c.evicted, k);
+}
+
+// Chunk-local keys carry the element's position 0..31 in their 5 low bits;
+// globalize swaps that for the 11-bit codeword index k0 + position.
+__device__ __forceinline__ float local_key(float s, int j) {
+    return __int_as_float((__float_as_int(s) & ~31) | j);
+}
+__device__ __forceinline__ float globalize(float k, int k0) {
+    const int b = __float_as_int(k);
+    return __int_as_float((b & ~0x7FF) | (k0 + (b & 31)));
+}
+
+// Best two of 32 keys: pairwise min/max, then a tree of top-2 merges.
+__device__ __forceinline__ void top2_of_32(const float (&k)[32], float& c1, float& c2) {
+    float L[16], H[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        L[i] = fminf(k[2 * i], k[2 * i + 1]);
+        H[i] = fmaxf(k[2 * i], k[2 * i + 1]);
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float a = L[2 * i], b = L[2 * i + 1];
+            L[i] = fminf(a, b);
+            H[i] = fmin3(fmaxf(a, b), H[2 * i], H[2 * i + 1]);
+        }
+    }
+    c1 = L[0];
+    c2 = H[0];
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -350,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         unsigned long long done = 0;
         long long p_tfull = 0, p_scan = 0, p_pick = 0, p_update = 0, p_stage = 0, p_esync = 0;
+        long long p_stmem = 0, p_smath = 0, p_spush = 0;
         long long t_mark = clock64();
         // attribute the cycles since the last mark to one counter
         auto mark = [&](long long& acc) {
@@ -503,8 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float twoE = 2.f * E;
                 Cands cs;
                 cands_reset(cs);
-                // raw scores above thr are outside the window of the best so far
-                float thr = __int_as_float(0x7f800000);
                 // ---- scan this half of the 16 score tiles of the codebook
                 for (int nt = 0; nt < NT; ++nt) {
                     const int bsel = tcnt & 1;
@@ -515,47 +550,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     uint32_t v[2][32];
+                    long long ts0 = clock64();
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64, v[0]);
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64 + 32, v[1]);
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
+                    long long ts1 = clock64();
+                    p_stmem += ts1 - ts0;
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
                         const int k0 = nt * BN + half * 64 + c2 * 32;
                         const float4* cn4 = reinterpret_cast<const float4*>(cn + k0);
-                        float sc[32];
+                        float kk[32];
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4) {
                             const float4 c = cn4[q4];
-                            sc[4 * q4 + 0] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 0]), c.x);
-                            sc[4 * q4 + 1] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 1]), c.y);
-                            sc[4 * q4 + 2] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 2]), c.z);
-                            sc[4 * q4 + 3] = fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w);
+                            kk[4 * q4 + 0] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 0]), c.x), 4 * q4 + 0);
+                            kk[4 * q4 + 1] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 1]), c.y), 4 * q4 + 1);
+                            kk[4 * q4 + 2] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 2]), c.z), 4 * q4 + 2);
+                            kk[4 * q4 + 3] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w), 4 * q4 + 3);
                         }
-                        float g[8];
+                        float c1k, c2k;
+                        top2_of_32(kk, c1k, c2k);
+                        ts0 = clock64();
+                        p_smath += ts0 - ts1;
+                        const float g1 = globalize(c1k, k0), g2 = globalize(c2k, k0);
+                        // the key that loses the best slot (or the chunk minimum, if it
+                        // does not take it) joins the list when it is inside the window
+                        const float dem = fmaxf(cs.best, g1);
+                        cs.best = fminf(cs.best, g1);
+                        const float thr = cs.best + key_slack(cs.best) + twoE;
+                        const float inf = __int_as_float(0x7f800000);
+                        cands_insert(cs, key_lower(dem) <= thr ? dem : inf);
+                        const bool second_in = key_lower(g2) <= thr;
+                        cands_insert(cs, second_in ? g2 : inf);
+                        if (second_in) {
+                            // rare: the chunk's third and later keys may be inside too
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
-                            g[q4] = fminf(fmin3(sc[4 * q4], sc[4 * q4 + 1], sc[4 * q4 + 2]),
-                                          sc[4 * q4 + 3]);
-                        const float cm = fminf(fmin3(g[0], g[1], g[2]),
-                                               fmin3(g[3], g[4], fmin3(g[5], g[6], g[7])));
-                        // the chunk minimum tightens the window before its groups are scanned
-                        thr = fminf(thr, cm + key_slack(cm) + twoE);
-                        if (cm <= thr) {
-#pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4) {
-                                if (g[q4] <= thr) {
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const float sv = sc[4 * q4 + e];
-                                        if (sv <= thr) cands_push(cs, make_key(sv, k0 + 4 * q4 + e));
-                                    }
-                                    thr = fminf(thr, cs.best + key_slack(cs.best) + twoE);
-                                }
+                            for (int j = 0; j < 32; ++j) {
+                                const float gj = globalize(kk[j], k0);
+                                const bool in = gj != g1 && gj != g2 && key_lower(gj) <= thr;
+                                cands_insert(cs, in ? gj : inf);
                             }
                         }
+                        ts1 = clock64();
+                        p_spush += ts1 - ts0;
                     }
                 }
                 if (!ok) break;
@@ -577,17 +618,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) cs.ts[p] = k0[p];
                     cs.best = k0[8];
-                    cs.evicted = k0[9];
+                    cs.evicted = fminf(k0[9], k1[9]);
                     const float best1 = k1[8];
-                    const float wthr0 = fminf(cs.best, best1);
-                    const float wthr = wthr0 + key_slack(wthr0) + twoE;
-                    cs.evicted = fminf(cs.evicted, k1[9]);
-#pragma unroll
-                    for (int p = 0; p < TOPK; ++p) {
-                        const float k = k1[p];
-                        if (key_lower(k) <= wthr) cands_push(cs, k);
-                    }
+                    cands_insert(cs, fmaxf(cs.best, best1));
                     cs.best = fminf(cs.best, best1);
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p) cands_insert(cs, k1[p]);
+                    cands_insert(cs, cs.best);  // the best heads the candidate list
+                    const float wthr = cs.best + key_slack(cs.best) + twoE;
                     int m = 0;
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) m += (key_lower(cs.ts[p]) <= wthr) ? 1 : 0;
@@ -724,6 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicAdd(prof + P_EPI_UPDATE, (unsigned long long)p_update);
             atomicAdd(prof + P_EPI_STAGE, (unsigned long long)p_stage);
             atomicAdd(prof + P_EPI_ESYNC, (unsigned long long)p_esync);
+            atomicAdd(prof + P_SCAN_TMEM, (unsigned long long)p_stmem);
+            atomicAdd(prof + P_SCAN_MATH, (unsigned long long)p_smath);
+            atomicAdd(prof + P_SCAN_PUSH, (unsigned long long)p_spush);
         }
         // count frames (one atomic per warp)
         for (int o = 16; o > 0; o >>= 1) done += __shfl_xor_sync(0xffffffffu, done, o);
