@@ -70,6 +70,12 @@ constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
 // ||bf16(r)|| ||bf16(c)||, twice the need), and the float32 score
 // ||c||^2 - 2 acc rounds once more (2^-21 of its magnitude, with slack).
 // E bounds |bf16 score - exact score| for every codeword.
+// Fine-grained timing of the scan loop (profile slots 12..14). Off by default:
+// the clock reads sit in the innermost loop.
+#ifndef MIMI_SCAN_TIMING
+#define MIMI_SCAN_TIMING 0
+#endif
+
 constexpr float kAccRel = 6.103515625e-05f;         // 2^-14
 constexpr float kScoreRel = 4.76837158203125e-07f;  // 2^-21
 
@@ -183,9 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
                 int* rescan_count, int* rescan_list, unsigned long long* stats,
                 unsigned long long* prof) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1 KiB alignment (128-byte swizzle atoms) as an offset into the shared
+    // array, so that the compiler keeps the shared address space (LDS / STS)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
     volatile int* abort = &bars->abort;
     const uint32_t ring = smem_u32(smem + RING_OFF);
@@ -550,14 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     uint32_t v[2][32];
-                    long long ts0 = clock64();
+                    long long ts0 = MIMI_SCAN_TIMING ? clock64() : 0;
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64, v[0]);
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64 + 32, v[1]);
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
-                    long long ts1 = clock64();
+                    long long ts1 = MIMI_SCAN_TIMING ? clock64() : 0;
                     p_stmem += ts1 - ts0;
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
@@ -574,8 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         float c1k, c2k;
                         top2_of_32(kk, c1k, c2k);
-                        ts0 = clock64();
-                        p_smath += ts0 - ts1;
+                        if (MIMI_SCAN_TIMING) {
+                            ts0 = clock64();
+                            p_smath += ts0 - ts1;
+                        }
                         const float g1 = globalize(c1k, k0), g2 = globalize(c2k, k0);
                         // the key that loses the best slot (or the chunk minimum, if it
                         // does not take it) joins the list when it is inside the window
@@ -587,16 +596,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool second_in = key_lower(g2) <= thr;
                         cands_insert(cs, second_in ? g2 : inf);
                         if (second_in) {
-                            // rare: the chunk's third and later keys may be inside too
+                            // the chunk's third and later keys may be inside too: count
+                            int cnt = 0;
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const float gj = globalize(kk[j], k0);
-                                const bool in = gj != g1 && gj != g2 && key_lower(gj) <= thr;
-                                cands_insert(cs, in ? gj : inf);
+                            for (int j = 0; j < 32; ++j) cnt += (key_lower(kk[j]) <= thr) ? 1 : 0;
+                            if (cnt > 2) {  // rare: insert every other key inside the window
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    const float gj = globalize(kk[j], k0);
+                                    const bool in = gj != g1 && gj != g2 && key_lower(gj) <= thr;
+                                    cands_insert(cs, in ? gj : inf);
+                                }
                             }
                         }
-                        ts1 = clock64();
-                        p_spush += ts1 - ts0;
+                        if (MIMI_SCAN_TIMING) {
+                            ts1 = clock64();
+                            p_spush += ts1 - ts0;
+                        }
                     }
                 }
                 if (!ok) break;
