@@ -352,37 +352,41 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_streaming(args):
-    """Per-call device latency of encode_step for B in {1, 16, 128, 1024}, 1000 calls each
-    (L2 flushed between calls when the inputs would fit in it)."""
+    """Per-call device latency of encode_step for B in {1, 16, 128, 1024}, 1000 calls each.
+    The calls cycle through a pool of distinct input batches larger than L2 (at least
+    256 MiB), so every call reads its frames from HBM; the codebook tables, which every call
+    reads, stay in L2 as they would in a streaming service."""
     import torch
     import split_residual_vector_b200 as pkg
     device = torch.device("cuda", 0)
     out = {}
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)  # 256 MiB > L2
     for B in (1, 16, 128, 1024):
         model, frames = synth.streaming_step(B, calls=args.calls)
         q = pkg.Quantizer(torch.from_numpy(model.C).to(device),
                           torch.from_numpy(model.W_in).to(device),
                           torch.from_numpy(model.W_out).to(device))
+        pool_calls = max(args.calls, (256 << 20) // (B * 512 * 4))
         f = torch.from_numpy(frames).to(device)
+        if pool_calls > args.calls:
+            reps = (pool_calls + args.calls - 1) // args.calls
+            f = f.repeat(reps, 1, 1)[:pool_calls].contiguous()
+        stride = 7919  # a prime step through the pool: consecutive calls touch distant batches
         codes = torch.empty((B, 8), dtype=torch.int16, device=device)
         stream = torch.cuda.current_stream(device)
         for i in range(5):
             q.encode_step(f[i], out=codes, stream=stream)
-        need_flush = frames.nbytes < (256 << 20)
         times = []
         for i in range(args.calls):
-            if need_flush:
-                flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            q.encode_step(f[i], out=codes, stream=stream)
+            q.encode_step(f[(i * stride) % f.shape[0]], out=codes, stream=stream)
             b.record(stream)
             times.append((a, b))
         torch.cuda.synchronize(device)
         ms = sorted(a.elapsed_time(b) for a, b in times)
         out[B] = {"median_us": 1e3 * ms[len(ms) // 2], "p99_us": 1e3 * ms[int(0.99 * len(ms))],
-                  "frames_per_s": B / (ms[len(ms) // 2] / 1e3), "l2_flushed": need_flush}
+                  "frames_per_s": B / (ms[len(ms) // 2] / 1e3),
+                  "input_pool_mib": f.numel() * 4 / 2**20}
         q.close()
     return {"metric": METRIC, "workload": f"streaming: {WORKLOADS['streaming']}",
             "calls": args.calls, "per_batch": out}

@@ -160,6 +160,21 @@ __device__ __forceinline__ float globalize(float k, int k0) {
     return __int_as_float((b & ~0x7FF) | (k0 + (b & 31)));
 }
 
+// min(1, max(0, a * b + c)) in one FMA-pipe instruction.
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+    float r;
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Smallest of 32 keys with a tree of 3-input minima (16 instructions).
+__device__ __forceinline__ float min_of_32(const float (&k)[32]) {
+    float m8[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m8[q] = fminf(fmin3(k[4 * q], k[4 * q + 1], k[4 * q + 2]), k[4 * q + 3]);
+    return fminf(fmin3(m8[0], m8[1], m8[2]), fmin3(m8[3], m8[4], fmin3(m8[5], m8[6], m8[7])));
+}
+
 // Best two of 32 keys: pairwise min/max, then a tree of top-2 merges.
 __device__ __forceinline__ void top2_of_32(const float (&k)[32], float& c1, float& c2) {
     float L[16], H[16];
@@ -579,32 +594,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                             kk[4 * q4 + 2] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 2]), c.z), 4 * q4 + 2);
                             kk[4 * q4 + 3] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w), 4 * q4 + 3);
                         }
-                        float c1k, c2k;
-                        top2_of_32(kk, c1k, c2k);
+                        const float c1k = min_of_32(kk);
                         if (MIMI_SCAN_TIMING) {
                             ts0 = clock64();
                             p_smath += ts0 - ts1;
                         }
-                        const float g1 = globalize(c1k, k0), g2 = globalize(c2k, k0);
+                        const float g1 = globalize(c1k, k0);
                         // the key that loses the best slot (or the chunk minimum, if it
                         // does not take it) joins the list when it is inside the window
                         const float dem = fmaxf(cs.best, g1);
                         cs.best = fminf(cs.best, g1);
                         const float thr = cs.best + key_slack(cs.best) + twoE;
                         const float inf = __int_as_float(0x7f800000);
-                        cands_insert(cs, key_lower(dem) <= thr ? dem : inf);
-                        const bool second_in = key_lower(g2) <= thr;
-                        cands_insert(cs, second_in ? g2 : inf);
-                        if (second_in) {
-                            // the chunk's third and later keys may be inside too: count
-                            int cnt = 0;
+                        const bool dem_in = key_lower(dem) <= thr;
+                        if (__any_sync(0xffffffffu, dem_in)) cands_insert(cs, dem_in ? dem : inf);
+                        // Any other key of the chunk inside the window? On the FMA pipe:
+                        // sum_j sat(kd (Td - key_j)), minus the minimum's own term. Td widens
+                        // thr by more than the key perturbations, and every key below Td adds
+                        // at least 2^-16, far above the rounding of the sum (<= 2^-18).
+                        const float Td = thr + 1.953125e-3f * (fabsf(thr) + twoE);
+                        const float kd = 16.f / (fabsf(Td) + twoE + 1e-30f);
+                        const float K = fmaf(kd, Td, 1.52587890625e-05f);
+                        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) cnt += (key_lower(kk[j]) <= thr) ? 1 : 0;
-                            if (cnt > 2) {  // rare: insert every other key inside the window
+                        for (int j = 0; j < 32; j += 4) {
+                            a0 += fma_sat(-kd, kk[j + 0], K);
+                            a1 += fma_sat(-kd, kk[j + 1], K);
+                            a2 += fma_sat(-kd, kk[j + 2], K);
+                            a3 += fma_sat(-kd, kk[j + 3], K);
+                        }
+                        const float other = ((a0 + a1) + (a2 + a3)) - fma_sat(-kd, c1k, K);
+                        const bool second_cand = other > 9.5367431640625e-07f;  // 2^-20
+                        if (__any_sync(0xffffffffu, second_cand)) {
+                            // some lane has another key near the window: its runner-up goes
+                            // in, and a third key is looked for only if the sum says so
+                            float c1b, c2k;
+                            top2_of_32(kk, c1b, c2k);
+                            const float g2 = globalize(c2k, k0);
+                            const bool second_in = second_cand && key_lower(g2) <= thr;
+                            cands_insert(cs, second_in ? g2 : inf);
+                            const bool more = second_cand &&
+                                              (other - fma_sat(-kd, c2k, K)) > 9.5367431640625e-07f;
+                            if (__any_sync(0xffffffffu, more)) {
 #pragma unroll
                                 for (int j = 0; j < 32; ++j) {
                                     const float gj = globalize(kk[j], k0);
-                                    const bool in = gj != g1 && gj != g2 && key_lower(gj) <= thr;
+                                    const bool in = more && gj != g1 && gj != g2 && key_lower(gj) <= thr;
                                     cands_insert(cs, in ? gj : inf);
                                 }
                             }
