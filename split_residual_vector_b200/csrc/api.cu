@@ -2,7 +2,7 @@
 //
 // Host side only: argument checks, the handle's device tables, TMA descriptor
 // encoding, and launches. Every step of the computation runs in the kernels of
-// prep.cu, encode_tc.cu, encode_scan.cu and decode.cu.
+// prep.cu, encode_tc.cu, encode_wide.cu, encode_scan.cu and decode.cu.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -76,7 +76,8 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 
 void free_tables(mimi::Tables& t) {
     void* ptrs[] = {t.C32, t.Win32, t.WinT32, t.Cbf, t.Win_hi, t.Win_lo, t.cnorm, t.cbound,
-                    t.P, t.err, t.rescan_count, t.rescan_list, t.stats};
+                    t.P, t.err, t.rescan_count, t.rescan_list, t.stats, t.wide_y,
+                    t.wide_bars, t.wide_partial};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     t = mimi::Tables{};
@@ -145,6 +146,12 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (e == cudaSuccess) e = dalloc(&t.rescan_count, 1);
     if (e == cudaSuccess) e = dalloc(&t.rescan_list, (size_t)mimi::kRescanCapacity);
     if (e == cudaSuccess) e = dalloc(&t.stats, 2);
+    if (e == cudaSuccess) e = dalloc(&t.wide_y, (size_t)mimi::kWideMaxFrames * kD);
+    if (e == cudaSuccess)
+        e = dalloc(&t.wide_bars, (size_t)mimi::kWideMaxGroups * mimi::kWideBarStride);
+    if (e == cudaSuccess)
+        e = cudaMalloc(reinterpret_cast<void**>(&t.wide_partial),
+                       mimi::wide_partial_bytes(h->num_sms));
     cudaStream_t s = nullptr;
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
     if (e == cudaSuccess)
@@ -154,10 +161,14 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (e == cudaSuccess) e = cudaMemsetAsync(t.err, 0, sizeof(int), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(t.rescan_count, 0, sizeof(int), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(t.stats, 0, 2 * sizeof(unsigned long long), s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(t.wide_bars, 0,
+                            sizeof(unsigned) * mimi::kWideMaxGroups * mimi::kWideBarStride, s);
     if (e == cudaSuccess) e = mimi::prep_tables(t, W_out, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (s) cudaStreamDestroy(s);
     if (e == cudaSuccess) e = mimi::encode_tc_configure();
+    if (e == cudaSuccess) e = mimi::encode_wide_configure();
     if (e != cudaSuccess) {
         free_tables(t);
         delete h;
@@ -214,7 +225,14 @@ int mimi_rvq_encode(mimi_rvq_t h, const void* latents, int dtype, int64_t N, int
 int mimi_rvq_encode_step(mimi_rvq_t h, const void* frames, int dtype, int B, int16_t* codes,
                          struct CUstream_st* stream) {
     if (B < 0) return MIMI_RVQ_EINVAL;
-    return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, kQ, 0, codes, stream);
+    if (!h) return MIMI_RVQ_EINVAL;
+    const mimi::WidePlan p = mimi::plan_encode_wide(B, h->num_sms);
+    if (!p.ok) return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, kQ, 0, codes, stream);
+    if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
+    const int c = check_common(h, frames, codes, B);
+    if (c <= 0) return c;
+    return from_cuda(
+        mimi::launch_encode_wide(h->t, p, frames, dtype, B, kQ, 0, codes, stream));
 }
 
 int mimi_rvq_encode_profile(mimi_rvq_t h, const void* latents, int dtype, int64_t N,
@@ -270,6 +288,11 @@ int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st* stream) {
     if (cudaMemcpy(&bits, h->t.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return MIMI_RVQ_ECUDA;
     if (bits && cudaMemset(h->t.err, 0, sizeof(int)) != cudaSuccess) return MIMI_RVQ_ECUDA;
+    // a wait that ran out may have left a group barrier mid-count
+    if ((bits & mimi::MIMI_DEV_ERR_TIMEOUT) &&
+        cudaMemset(h->t.wide_bars, 0,
+                   sizeof(unsigned) * mimi::kWideMaxGroups * mimi::kWideBarStride) != cudaSuccess)
+        return MIMI_RVQ_ECUDA;
     if (bits & mimi::MIMI_DEV_ERR_TIMEOUT) return MIMI_RVQ_ETIMEOUT;
     if (bits & mimi::MIMI_DEV_ERR_RANGE) return MIMI_RVQ_ERANGE;
     return MIMI_RVQ_OK;

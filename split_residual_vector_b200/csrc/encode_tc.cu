@@ -83,10 +83,8 @@ constexpr float kScoreRel = 4.76837158203125e-07f;  // 2^-21
 // the codeword index, so that one min/max orders (score, index) pairs and the
 // index travels with the score. The replacement moves the value by less than
 // 2^-12 of its magnitude; every comparison that must be rigorous widens by
-// key_slack(x) = 2^-11 |x|, which covers it.
-__device__ __forceinline__ float make_key(float s, int idx) {
-    return __int_as_float((__float_as_int(s) & ~0x7FF) | idx);
-}
+// key_slack(x) = 2^-11 |x|, which covers it. Keys are built in two steps
+// (local_key, then globalize) below.
 __device__ __forceinline__ int key_index(float k) { return __float_as_int(k) & 0x7FF; }
 __device__ __forceinline__ float key_slack(float k) { return fabsf(k) * 4.8828125e-4f; }
 // Smallest raw score a key can stand for (an empty slot, +inf, stays +inf).

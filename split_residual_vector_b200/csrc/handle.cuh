@@ -19,6 +19,15 @@ constexpr int kQ = 8;         // codebooks: 0 semantic, 1..7 acoustic
 // list cannot overflow).
 constexpr int64_t kRescanCapacity = 1 << 20;
 
+// Largest streaming step the latency (wide) encoder takes; larger steps go to
+// the tensor-core encoder, which is as fast from about 900 frames up (measured
+// per-call latency on B200: 54 us at 1 frame, 121 us at 128, 318 us at 768,
+// 392 us at 1024, against 290-380 us for the tensor-core encoder).
+constexpr int kWideMaxFrames = 896;
+constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
+constexpr int kWideMaxGroups = 64;    // group barriers
+constexpr int kWideBarStride = 32;    // words per group barrier (count, generation; own 128 B line)
+
 struct Tables {
     // float32 originals
     float* C32 = nullptr;         // [Q][K][D] codebooks (0 semantic)
@@ -36,6 +45,9 @@ struct Tables {
     int* rescan_count = nullptr;      // frames queued for the full scan in this launch
     int* rescan_list = nullptr;       // [kRescanCapacity] frame indices
     unsigned long long* stats = nullptr;  // [0] frames encoded, [1] frames re-scanned
+    float* wide_y = nullptr;          // [kWideMaxFrames][D] latency encoder: projection exchange
+    unsigned* wide_bars = nullptr;                // [kWideMaxGroups][kWideBarStride] group barriers
+    unsigned long long* wide_partial = nullptr;   // per-CTA minimum keys, wide_partial_bytes()
     // TMA descriptors (bf16, 64 x 128 boxes, 128-byte swizzle)
     CUtensorMap tm_C;             // Cbf as [Q*K rows][D cols]
     CUtensorMap tm_Whi;           // Win_hi as [D rows][Din cols]
@@ -57,6 +69,23 @@ cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_
                                int variant, int16_t* codes, cudaStream_t s);
 cudaError_t launch_rescan(const Tables& t, const void* z, int dtype, int n_q, int variant,
                           int16_t* codes, cudaStream_t s);
+// encode_wide.cu
+struct WidePlan {
+    bool ok = false;   // false: B is outside (0, kWideMaxFrames] or needs more CTAs than SMs
+    int groups = 0;    // frame groups of at most 64
+    int S = 0;         // CTAs per group (codebook slices)
+    int per_k = 0;     // codewords per slice
+    int grid = 0;      // groups * S (<= SM count: every CTA resident at once)
+    int U = 0, V = 0;  // thread tile: 16U frames x 16V codewords
+    int jc = 0;        // projection: latent columns staged per pass
+    int smem = 0;      // dynamic shared memory bytes
+};
+WidePlan plan_encode_wide(int B, int num_sms);
+size_t wide_partial_bytes(int num_sms);
+cudaError_t encode_wide_configure();  // once per device, before the first launch
+// Launches on one set of tables must be stream-ordered (they share the scratch).
+cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z, int dtype, int B,
+                               int n_q, int variant, int16_t* codes, cudaStream_t s);
 // decode.cu
 cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int n_q, float* out,
                           cudaStream_t s);

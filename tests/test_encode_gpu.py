@@ -128,6 +128,64 @@ def test_streaming_step(batch):
     assert q.get_error() == 0
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_streaming_step_equals_full_scan(dtype):
+    """Small steps run the latency encoder, whose scores are the float32 full scan's
+    (same sums in the same order): every code equals encode_scan's, near ties included.
+    Sizes span one to 64 frame groups, ragged group tails and every thread-tile shape."""
+    model, frames = synth.streaming_step(896, calls=1)
+    q = quantizer(model)
+    z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
+    zd = to_device(np.ascontiguousarray(z))
+    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 833, 896)
+    for b in sizes:
+        step = q.encode_step(zd[:b]).cpu().numpy()
+        scan = q.encode_scan(zd[:b]).cpu().numpy()
+        assert np.array_equal(step, scan), f"B={b}: {np.argwhere(step != scan)[:5]}"
+    enc, _ = q.stats()
+    assert enc == sum(sizes)
+    assert q.get_error() == 0
+
+
+@pytest.mark.parametrize("batch", [897, 1024, 5000])
+def test_streaming_step_large_batch_uses_the_batch_encoder(batch):
+    """Above the latency encoder's batch limit (896) a step is a batch encode."""
+    model, frames = synth.streaming_step(batch, calls=1)
+    q = quantizer(model)
+    codes = q.encode_step(to_device(np.ascontiguousarray(frames[0]))).cpu().numpy()
+    idx = np.concatenate([np.arange(0, 200), np.arange(batch - 100, batch)])
+    ref, db, ds = oracle.encode(frames[0][idx], model.W_in, model.C)
+    assert_codes_match(codes[idx], ref, db, ds, f"step B={batch}")
+    assert q.get_error() == 0
+
+
+@pytest.mark.parametrize("batch", [1, 128])
+def test_streaming_step_in_a_cuda_graph(batch):
+    """The latency encoder's group barriers return to their starting state after every
+    launch, so a captured step replays correctly on new inputs."""
+    model, frames = synth.streaming_step(batch, calls=4)
+    q = quantizer(model)
+    static_in = to_device(np.ascontiguousarray(frames[0]))
+    static_out = torch.empty((batch, 8), dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        q.encode_step(static_in, out=static_out, stream=s)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        q.encode_step(static_in, out=static_out, stream=torch.cuda.current_stream())
+    for call in range(4):
+        static_in.copy_(to_device(np.ascontiguousarray(frames[call])))
+        g.replay()
+        torch.cuda.synchronize()
+        got = static_out.cpu().numpy()
+        want = q.encode_scan(static_in).cpu().numpy()
+        assert np.array_equal(got, want), f"replay {call}"
+    assert q.get_error() == 0
+
+
 # ------------------------------------------------------------------ adversarial inputs
 
 
