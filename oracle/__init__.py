@@ -7,7 +7,9 @@ two share no code: this module only marshals numpy arrays into the plain C in
 
 What it computes, and the passages it follows, is documented in ``oracle.c``:
 y = W_in z (512 -> 256), a semantic plain VQ on y, a greedy 7-level acoustic
-RVQ on y, codes (s, a_1..a_7); decode = W_out (S_s + sum_l A_{l,a_l}).
+RVQ on y, codes (s, a_1..a_7); decode = W_out (S_s + sum_l A_{l,a_l}); and in
+``moshi_streams.c``: the delay-pattern packing of the 17-stream frame, its
+inverse, and the sum of per-stream embeddings that feeds the language model.
 """
 from __future__ import annotations
 
@@ -16,7 +18,7 @@ import os
 
 import numpy as np
 
-from .build import build_oracle, library_path
+from .build import build_oracle, library_path, sources
 
 F32, BF16 = 0, 1
 NEAR_TIE_REL = 1e-5  # gap <= 1e-5 * (1 + d_best) at some level marks a near-tie frame
@@ -29,8 +31,8 @@ def _load():
     if _lib is not None:
         return _lib
     path = library_path()
-    src = os.path.join(os.path.dirname(__file__), "oracle.c")
-    if not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(src):
+    if not os.path.exists(path) or os.path.getmtime(path) < max(os.path.getmtime(f)
+                                                                 for f in sources()):
         build_oracle()
     lib = ctypes.CDLL(path)
     c_i64, c_int, c_vp, c_dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_double
@@ -53,6 +55,16 @@ def _load():
     lib.oracle_bitrate.restype = c_dbl
     lib.oracle_threads.argtypes = [c_int]
     lib.oracle_threads.restype = c_int
+    lib.oracle_delay_pack.argtypes = [c_vp, c_vp, c_int, c_i64, c_int, c_vp, c_i64,
+                                      ctypes.c_int32, ctypes.c_int32, c_vp]
+    lib.oracle_delay_pack.restype = c_int
+    lib.oracle_delay_unpack.argtypes = [c_vp, c_i64, c_int, c_int, c_int, c_vp, c_i64, c_vp]
+    lib.oracle_delay_unpack.restype = c_int
+    lib.oracle_delay_latency_ms.argtypes = [c_vp, c_int, c_dbl]
+    lib.oracle_delay_latency_ms.restype = c_dbl
+    lib.oracle_embed_sum.argtypes = [c_vp, c_int, c_int, c_vp, c_int, c_vp, c_i64, c_int, c_vp,
+                                     c_vp]
+    lib.oracle_embed_sum.restype = c_int
     _lib = lib
     return lib
 
@@ -178,3 +190,64 @@ def bits_per_code(K: int) -> int:
 
 def bitrate(frame_rate_hz: float, Q: int, K: int) -> float:
     return float(_load().oracle_bitrate(float(frame_rate_hz), int(Q), int(K)))
+
+
+# ----------------------------------------------------------------- Moshi token streams
+
+TEXT_CARD, AUDIO_CARD = 32000, 2048
+TEXT_PAD, AUDIO_PAD = TEXT_CARD, AUDIO_CARD  # pad ids: one past each vocabulary
+
+
+def delay_pack(text, audio, delays, S: int | None = None, text_pad: int = TEXT_PAD,
+               audio_pad: int = AUDIO_PAD) -> np.ndarray:
+    """Multi-stream frame V [S, 1 + n_audio * Q] int32 from text [T] int32 (or None) and
+    audio [n_audio, T, Q] int16 with per-level delays [Q]. S defaults to T + max delay."""
+    lib = _load()
+    audio = np.ascontiguousarray(audio, dtype=np.int16)
+    n_audio, T, Q = audio.shape
+    d = np.ascontiguousarray(delays, dtype=np.int32)
+    assert d.shape == (Q,)
+    S = T + int(d.max(initial=0)) if S is None else int(S)
+    t = None if text is None else np.ascontiguousarray(text, dtype=np.int32)
+    assert t is None or t.shape == (T,)
+    V = np.empty((S, 1 + n_audio * Q), np.int32)
+    _check(lib.oracle_delay_pack(_ptr(t), _ptr(audio), n_audio, T, Q, _ptr(d), S, text_pad,
+                                 audio_pad, _ptr(V)), "delay_pack")
+    return V
+
+
+def delay_unpack(V, col0: int, delays, T: int | None = None) -> np.ndarray:
+    """audio [T, Q] int16 from the Q columns of V starting at col0 (inverse of the shift).
+    T defaults to S - max delay."""
+    lib = _load()
+    V = np.ascontiguousarray(V, dtype=np.int32)
+    S, K = V.shape
+    d = np.ascontiguousarray(delays, dtype=np.int32)
+    Q = d.shape[0]
+    T = S - int(d.max(initial=0)) if T is None else int(T)
+    out = np.empty((T, Q), np.int16)
+    _check(lib.oracle_delay_unpack(_ptr(V), S, K, col0, Q, _ptr(d), T, _ptr(out)),
+           "delay_unpack")
+    return out
+
+
+def delay_latency_ms(delays, frame_ms: float = 80.0) -> float:
+    d = np.ascontiguousarray(delays, dtype=np.int32)
+    return float(_load().oracle_delay_latency_ms(_ptr(d), len(d), float(frame_ms)))
+
+
+def embed_sum(tables, rows, V, nthreads: int = 0):
+    """out [S, d] float64 = sum over k of row V[s, k] of table k; returns (out, n_bad).
+    tables: the K tables' rows stacked [sum(rows), d], float32 or bf16 bit patterns (uint16)."""
+    lib = _load()
+    tables, dt = _latents(tables)
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+    V = np.ascontiguousarray(V, dtype=np.int32)
+    S, K = V.shape
+    assert r.shape == (K,) and tables.shape[0] == int(r.sum())
+    d = tables.shape[1]
+    out = np.empty((S, d), np.float64)
+    bad = np.zeros(1, np.int64)
+    _check(lib.oracle_embed_sum(_ptr(tables), dt, K, _ptr(r), d, _ptr(V), S, nthreads, _ptr(out),
+                                _ptr(bad)), "embed_sum")
+    return out, int(bad[0])

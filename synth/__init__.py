@@ -13,6 +13,9 @@ of 2048, codebook 0 semantic, 1..7 acoustic):
 * ``streaming_step``  -- B concurrent streams, one fp32 frame each, 1000 calls;
 * ``bulk_tokenization`` -- 1 048 576 bf16 frames, encode only;
 * ``decode_heavy``    -- 1 048 576 frames of codes (semantic uniform, acoustic Zipf(1.1)).
+* ``moshi_input``     -- the language model's side of the codec: text tokens and two audio
+  code streams (Moshi, user) of T frames, and 17 embedding tables (text 32 000 + 1 rows,
+  16 audio tables of 2048 + 1 rows; the extra row is the pad token), d = 4096, bf16.
 
 Generation recipe: W_in ~ N(0, 1/512) [256, 512]; W_out ~ N(0, 1/256) [512, 256];
 S ~ N(0, 1) [2048, 256]; A_l ~ N(0, 0.5^(2l)) [2048, 256] for l = 1..7; latents
@@ -168,3 +171,35 @@ def decode_heavy(n: int = 1 << 20, seed: int = 4):
     codes[:, 0] = rng.integers(0, K, size=n).astype(np.int16)
     codes[:, 1:] = zipf_codes(rng, (n, Q - 1))
     return model, codes
+
+
+TEXT_CARD, AUDIO_CARD, MOSHI_DIM = 32000, 2048, 4096
+
+
+def moshi_streams(T: int, seed: int = 5, n_audio: int = 2):
+    """text [T] int32 uniform on [0, 32000); audio [n_audio, T, 8] int16 with level 0
+    uniform on [0, 2048) and levels 1..7 Zipf(1.1) (the decode-heavy code statistics)."""
+    rng = generator(seed)
+    text = rng.integers(0, TEXT_CARD, size=T).astype(np.int32)
+    audio = np.empty((n_audio, T, Q), np.int16)
+    for a in range(n_audio):
+        audio[a, :, 0] = rng.integers(0, K, size=T).astype(np.int16)
+        audio[a, :, 1:] = zipf_codes(rng, (T, Q - 1))
+    return text, audio
+
+
+def moshi_rows(n_audio: int = 2):
+    """Row counts of the stacked embedding tables: text, then n_audio x 8 audio tables."""
+    return [TEXT_CARD + 1] + [AUDIO_CARD + 1] * (n_audio * Q)
+
+
+def moshi_tables(d: int = MOSHI_DIM, seed: int = 6, n_audio: int = 2, rows=None) -> np.ndarray:
+    """Stacked embedding tables [sum(rows), d] as bf16 bit patterns, entries N(0, 1)."""
+    rng = generator(seed)
+    rows = moshi_rows(n_audio) if rows is None else rows
+    out = np.empty((int(sum(rows)), d), np.uint16)
+    step = max(1, (1 << 24) // d)
+    for r0 in range(0, out.shape[0], step):
+        r1 = min(out.shape[0], r0 + step)
+        out[r0:r1] = to_bf16_bits(normal(rng, (r1 - r0, d)))
+    return out
