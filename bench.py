@@ -45,6 +45,16 @@ WORKLOADS = {
     "decode_heavy": "1048576 frames of codes (semantic uniform, acoustic Zipf(1.1)); decode "
                     "to fp32 [1048576,512]",
     "streaming": "B concurrent streams, one fp32 frame each per call; encode_step",
+    "moshi_input": "65536 frames of Moshi + user codes (semantic uniform, acoustic Zipf(1.1)) "
+                   "and text tokens (uniform over 32000); delay-pattern packing with tau = 1 "
+                   "into 17 streams, then the sum of 17 bf16 embedding tables (text 32001 rows, "
+                   "16 x 2049 audio rows, d = 4096) per step, bf16 out [65537,4096]",
+}
+MOSHI_DELAYS = [0, 1, 1, 1, 1, 1, 1, 1]   # acoustic delay 1 (the final model's)
+# DRAM bytes (read + write) per unit from one ncu capture of the current kernel, with the
+# summary that records it; the bench scales it by the units of a launch. None: not captured.
+NCU_TRAFFIC_PER_UNIT = {
+    "k_embed_sum": (48_951, "profiles/k_embed_sum_moshi_input.md"),   # per step
 }
 
 
@@ -71,27 +81,42 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu_index = gpu_index
         self.proc = None
+        self.lines = []
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append(ln)
+                self.started.set()
 
     def __enter__(self):
+        import threading
+        self.started = threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.gpu_index)],
+                 "-lms", "50", "-i", str(self.gpu_index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        self.started.wait(timeout=10)  # sampling is live before the timed region starts
+        self.lines.clear()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
+            import time as _t
+            _t.sleep(0.06)  # one more sample interval covers the end of the region
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=10)
+                self.proc.wait(timeout=10)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=10)
         return False
 
     def summary(self):
@@ -392,6 +417,167 @@ def run_streaming(args):
             "calls": args.calls, "per_batch": out}
 
 
+def run_moshi_input(args, rank, world, local_rank):
+    """The language model's side of the codec: pack + embedding sum (one step = both calls
+    over the whole workload)."""
+    import torch
+    import split_residual_vector_b200 as pkg
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    T = args.frames or (1 << 16)
+    text_h, audio_h = synth.moshi_streams(T, seed=5 + 100 * rank)
+    rows = synth.moshi_rows()
+    tables_h = synth.moshi_tables(seed=6 + 100 * rank)
+    d = tables_h.shape[1]
+    K = len(rows)
+    S = T + max(MOSHI_DELAYS)
+    text = torch.from_numpy(text_h).to(device)
+    audio = torch.from_numpy(audio_h).to(device)
+    tables = torch.from_numpy(tables_h.view(np.int16)).to(device).view(torch.bfloat16)
+    packed = torch.empty((S, K), dtype=torch.int32, device=device)
+    out = torch.empty((S, d), dtype=torch.bfloat16, device=device)
+    n_bad = torch.zeros(1, dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream(device)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    pack_ms, emb_ms = [], []
+
+    def step(timed):
+        a, b, c = ev(), ev(), ev()
+        a.record(stream)
+        pkg.delay_pack(text, audio, MOSHI_DELAYS, out=packed, stream=stream)
+        b.record(stream)
+        pkg.embed_sum(tables, rows, packed, out=out, n_bad=n_bad, stream=stream)
+        c.record(stream)
+        if timed:
+            pack_ms.append((a, b))
+            emb_ms.append((b, c))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    start, stop = ev(), ev()
+    with ClockSampler(local_rank) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    elapsed_ms = start.elapsed_time(stop)
+    if dist:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = T * world / (ms_per_step / 1e3)
+    pack_avg = sum(a.elapsed_time(b) for a, b in pack_ms) / len(pack_ms)
+    emb_avg = sum(a.elapsed_time(b) for a, b in emb_ms) / len(emb_ms)
+    bad = int(n_bad.item())
+
+    e2e = None
+    if not args.no_e2e:
+        k = max(3, min(args.steps, 5))
+        h_text = torch.empty_like(text, device="cpu").pin_memory()
+        h_audio = torch.empty_like(audio, device="cpu").pin_memory()
+        h_text.copy_(text)
+        h_audio.copy_(audio)
+        h_out = torch.empty((S, d), dtype=torch.bfloat16, pin_memory=True)
+
+        def e2e_step():
+            text.copy_(h_text, non_blocking=True)
+            audio.copy_(h_audio, non_blocking=True)
+            pkg.delay_pack(text, audio, MOSHI_DELAYS, out=packed, stream=stream)
+            pkg.embed_sum(tables, rows, packed, out=out, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if dist:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(k):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = a.elapsed_time(b) / k
+        if dist:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": T * world / (e_ms / 1e3), "unit": "frames/s",
+               "h2d_bytes_per_step": text.numel() * 4 + audio.numel() * 2,
+               "d2h_bytes_per_step": out.numel() * 2, "ms_per_step": e_ms, "steps": k}
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return None
+    peaks = load_peaks()
+    row_bytes = d * 2
+    emb_bytes = K * row_bytes + K * 4 + row_bytes   # gathered rows + tokens + bf16 out, per step
+    pack_bytes = 4 + 2 * 8 * 2 + K * 4              # text + codes in, packed row out, per step
+    emb_gbs = emb_bytes * S / (emb_avg / 1e3) / 1e9
+    pack_gbs = pack_bytes * S / (pack_avg / 1e3) / 1e9
+    kernels = [
+        {"kernel": "k_embed_sum", "bound": "hbm", "achieved": emb_gbs, "peak": peaks["hbm_gbs"],
+         "unit": "GB/s", "frac": emb_gbs / peaks["hbm_gbs"],
+         "traffic": NCU_TRAFFIC_PER_UNIT["k_embed_sum"][0] * S,
+         "traffic_source": NCU_TRAFFIC_PER_UNIT["k_embed_sum"][1],
+         "dram_gbs_from_traffic": NCU_TRAFFIC_PER_UNIT["k_embed_sum"][0] * S / (emb_avg / 1e3) / 1e9,
+         "ms": emb_avg,
+         "algorithmic": f"{emb_bytes} B/step ({K} gathered bf16 rows of {d}, tokens, bf16 out) "
+                        f"x {S} steps; hot rows may come from L2"},
+        {"kernel": "k_delay_pack", "bound": "hbm", "achieved": pack_gbs, "peak": peaks["hbm_gbs"],
+         "unit": "GB/s", "frac": pack_gbs / peaks["hbm_gbs"], "traffic": None, "ms": pack_avg,
+         "algorithmic": f"{pack_bytes} B/step x {S} steps"}]
+    roofline = {k: kernels[0][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = "k_embed_sum"
+    roofline["peak_source"] = f"{peaks['source']} hbm_gbs"
+    line = {
+        "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 tables, f32 accumulate, bf16 out; int32 tokens", "data": "synthetic",
+        "config": {"workload": f"moshi_input: {WORKLOADS['moshi_input']}"
+                               + (f" (reduced to {T} frames)" if args.frames else ""),
+                   "frames_per_gpu": T, "steps_per_frame_stream": S, "delays": MOSHI_DELAYS,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "output (537 MB) larger than L2; tables 531 MB, hot rows stay in L2"},
+        "realtime_streams": value / FRAME_HZ, "roofline": roofline, "kernels": kernels,
+        "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "status": 0 if bad == 0 else -4,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        cores = oracle.threads(0)
+        n = 256
+        for _ in range(2):
+            t0 = time.perf_counter()
+            V = oracle.delay_pack(text_h[:n], audio_h[:, :n], MOSHI_DELAYS)
+            oracle.embed_sum(tables_h, rows, V)
+            dt = time.perf_counter() - t0
+            if dt > 3.0:
+                break
+            n = int(min(T, n * 12.0 / max(dt, 1e-3)))
+        line["cpu_baseline"] = {"value": n / dt, "unit": "frames/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"first {n} frames: pack + embedding sum, float64 "
+                                          f"oracle, {dt:.1f} s"}
+    if dist:
+        dist.destroy_process_group()
+    return line
+
+
 # --------------------------------------------------------------------- reference arm
 
 
@@ -399,11 +585,23 @@ def run_reference(args):
     """The float64 oracle on the host cores, each step a bounded sample of the workload."""
     import oracle
     name = args.workload
-    work = make_workload(name, 0)
-    m = work["model"]
+    if name == "moshi_input":
+        text_h, audio_h = synth.moshi_streams(args.frames or (1 << 16), seed=5)
+        tables_h, rows = synth.moshi_tables(seed=6), synth.moshi_rows()
+        work = {"frames": len(text_h)}
+    elif name == "streaming":
+        model, frames = synth.streaming_step(1024, calls=1)
+        work = {"model": model, "z": frames[0], "frames": frames.shape[1]}
+    else:
+        work = make_workload(name, 0)
 
     def one(nf):
-        if name in ("offline_batch", "bulk_tokenization"):
+        if name == "moshi_input":
+            oracle.embed_sum(tables_h, rows,
+                             oracle.delay_pack(text_h[:nf], audio_h[:, :nf], MOSHI_DELAYS))
+            return
+        m = work["model"]
+        if name in ("offline_batch", "bulk_tokenization", "streaming"):
             c, _, _ = oracle.encode(work["z"][:nf], m.W_in, m.C)
             if name == "offline_batch":
                 oracle.decode(c, m.C, m.W_out)
@@ -465,7 +663,10 @@ def main():
         if rank == 0:
             print(json.dumps(run_streaming(args)), flush=True)
         return
-    line = run_ours(args, rank, world, local_rank)
+    if args.workload == "moshi_input":
+        line = run_moshi_input(args, rank, world, local_rank)
+    else:
+        line = run_ours(args, rank, world, local_rank)
     if line is not None:
         print(json.dumps(line), flush=True)
 

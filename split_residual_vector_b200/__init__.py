@@ -22,7 +22,9 @@ LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmimi
 EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_encode_ex",
            "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
            "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror",
-           "mimi_rvq_encode_profile")
+           "mimi_rvq_encode_profile", "mimi_rvq_delay_pack", "mimi_rvq_delay_unpack",
+           "mimi_rvq_embed_sum")
+TEXT_CARD, TEXT_PAD, AUDIO_PAD = 32000, 32000, 2048
 
 _lib = None
 
@@ -68,6 +70,13 @@ def library() -> ctypes.CDLL:
     lib.mimi_rvq_stats.restype = ci
     lib.mimi_rvq_strerror.argtypes = [ci]
     lib.mimi_rvq_strerror.restype = ctypes.c_char_p
+    i32 = ctypes.c_int32
+    lib.mimi_rvq_delay_pack.argtypes = [vp, vp, ci, i64, vp, i64, i32, i32, vp, vp]
+    lib.mimi_rvq_delay_pack.restype = ci
+    lib.mimi_rvq_delay_unpack.argtypes = [vp, i64, ci, ci, vp, i64, vp, vp]
+    lib.mimi_rvq_delay_unpack.restype = ci
+    lib.mimi_rvq_embed_sum.argtypes = [vp, ci, ci, vp, ci, vp, i64, vp, ci, vp, vp]
+    lib.mimi_rvq_embed_sum.restype = ci
     _lib = lib
     return lib
 
@@ -223,3 +232,73 @@ class Quantizer:
         _check(library().mimi_rvq_stats(self._h, _stream(stream), ctypes.byref(a),
                                         ctypes.byref(b)), "mimi_rvq_stats")
         return a.value, b.value
+
+
+# ----------------------------------------------------------------- token streams
+
+
+def _host_i32(values, n):
+    arr = (ctypes.c_int32 * n)(*[int(v) for v in values])
+    assert len(values) == n
+    return arr
+
+
+def delay_pack(text, audio, delays, S=None, text_pad=TEXT_PAD, audio_pad=AUDIO_PAD, out=None,
+               stream=None):
+    """Multi-stream sequence [S, 1 + 8 * n_audio] int32 from text [T] int32 (or None) and
+    audio codes [n_audio, T, 8] int16 (CUDA), level q shifted later by delays[q] steps.
+    S defaults to T + max(delays)."""
+    import torch
+    assert audio.dtype == torch.int16 and audio.dim() == 3 and audio.shape[2] == NUM_CODEBOOKS
+    assert audio.is_contiguous()
+    n_audio, T, _ = audio.shape
+    S = T + max(int(v) for v in delays) if S is None else int(S)
+    K = 1 + NUM_CODEBOOKS * n_audio
+    if text is not None:
+        assert text.dtype == torch.int32 and text.is_contiguous() and text.shape == (T,)
+    if out is None:
+        out = torch.empty((S, K), dtype=torch.int32, device=audio.device)
+    assert out.dtype == torch.int32 and out.is_contiguous() and out.shape == (S, K)
+    _check(library().mimi_rvq_delay_pack(None if text is None else text.data_ptr(),
+                                         audio.data_ptr(), n_audio, T,
+                                         _host_i32(delays, NUM_CODEBOOKS), S, int(text_pad),
+                                         int(audio_pad), out.data_ptr(), _stream(stream)),
+           "mimi_rvq_delay_pack")
+    return out
+
+
+def delay_unpack(packed, col0, delays, T=None, out=None, stream=None):
+    """Audio codes [T, 8] int16 from the 8 columns of packed [S, K] int32 that start at col0
+    (the inverse shift). T defaults to S - max(delays)."""
+    import torch
+    assert packed.dtype == torch.int32 and packed.dim() == 2 and packed.is_contiguous()
+    S, K = packed.shape
+    T = S - max(int(v) for v in delays) if T is None else int(T)
+    if out is None:
+        out = torch.empty((T, NUM_CODEBOOKS), dtype=torch.int16, device=packed.device)
+    assert out.dtype == torch.int16 and out.is_contiguous() and out.shape == (T, NUM_CODEBOOKS)
+    _check(library().mimi_rvq_delay_unpack(packed.data_ptr(), S, K, int(col0),
+                                           _host_i32(delays, NUM_CODEBOOKS), T, out.data_ptr(),
+                                           _stream(stream)), "mimi_rvq_delay_unpack")
+    return out
+
+
+def embed_sum(tables, rows, tokens, out_dtype=None, out=None, n_bad=None, stream=None):
+    """out [S, d] = sum over k of row tokens[s, k] of table k. tables: stacked rows
+    [sum(rows), d] float32 / bfloat16 (CUDA); rows: the K row counts; tokens [S, K] int32.
+    n_bad: optional CUDA int64 [1] (caller-zeroed) counting tokens past their table."""
+    import torch
+    assert tables.dim() == 2 and tables.is_contiguous()
+    assert tokens.dtype == torch.int32 and tokens.dim() == 2 and tokens.is_contiguous()
+    S, K = tokens.shape
+    d = tables.shape[1]
+    assert len(rows) == K and sum(int(r) for r in rows) == tables.shape[0]
+    if out is None:
+        out = torch.empty((S, d), dtype=out_dtype or tables.dtype, device=tables.device)
+    assert out.is_contiguous() and out.shape == (S, d)
+    host_rows = (ctypes.c_int64 * K)(*[int(r) for r in rows])
+    _check(library().mimi_rvq_embed_sum(tables.data_ptr(), _dtype_flag(tables), K, host_rows, d,
+                                        tokens.data_ptr(), S, out.data_ptr(), _dtype_flag(out),
+                                        None if n_bad is None else n_bad.data_ptr(),
+                                        _stream(stream)), "mimi_rvq_embed_sum")
+    return out
