@@ -100,7 +100,7 @@ int mimi_rvq_encode(mimi_rvq_t h, const void *latents, int dtype, int64_t N,
 /*
  * Streaming step: one 512-d frame for each of B concurrent streams (B >= 0),
  * frames [B][512] -> codes [B][8]. The quantiser keeps no state between
- * frames, so a step is an encode of B frames tuned for latency: up to 896
+ * frames, so a step is an encode of B frames tuned for latency: up to 1024
  * frames run a float32 kernel spread over every SM (its codes equal
  * mimi_rvq_encode_scan's), larger steps run the batch encoder. Allocates
  * nothing, never synchronises the host, and may be captured in a CUDA graph.

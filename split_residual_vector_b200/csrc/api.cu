@@ -88,6 +88,16 @@ cudaError_t dalloc(T** p, size_t count) {
     return cudaMalloc(reinterpret_cast<void**>(p), sizeof(T) * count);
 }
 
+// Re-encode the frames the tensor-core kernel queued (count on the device) with
+// the float32 wide encoder, 1024 frames at a time.
+cudaError_t rescan(mimi_rvq_t h, const void* z, int dtype, int n_q, int variant, int16_t* codes,
+                   cudaStream_t s) {
+    const mimi::WidePlan p = mimi::plan_encode_wide(mimi::kWideMaxFrames, h->num_sms);
+    if (!p.ok) return cudaErrorInvalidConfiguration;
+    return mimi::launch_encode_wide(h->t, p, z, dtype, mimi::kWideMaxFrames, n_q, variant, codes,
+                                    s, true);
+}
+
 int check_common(mimi_rvq_t h, const void* in, const void* out, int64_t n) {
     if (!h || n < 0) return MIMI_RVQ_EINVAL;
     if (n == 0) return MIMI_RVQ_OK;
@@ -211,7 +221,7 @@ int mimi_rvq_encode_ex(mimi_rvq_t h, const void* latents, int dtype, int64_t N, 
         if (e == cudaSuccess)
             e = mimi::launch_encode_tc(h->t, z, dtype, n, n_q, variant, out, nullptr, stream,
                                        h->num_sms);
-        if (e == cudaSuccess) e = mimi::launch_rescan(h->t, z, dtype, n_q, variant, out, stream);
+        if (e == cudaSuccess) e = rescan(h, z, dtype, n_q, variant, out, stream);
         if (e != cudaSuccess) return from_cuda(e);
     }
     return MIMI_RVQ_OK;
@@ -246,7 +256,7 @@ int mimi_rvq_encode_profile(mimi_rvq_t h, const void* latents, int dtype, int64_
     if (e == cudaSuccess)
         e = mimi::launch_encode_tc(h->t, latents, dtype, N, kQ, 0, codes, nullptr, stream,
                                    h->num_sms, reinterpret_cast<unsigned long long*>(cycles));
-    if (e == cudaSuccess) e = mimi::launch_rescan(h->t, latents, dtype, kQ, 0, codes, stream);
+    if (e == cudaSuccess) e = rescan(h, latents, dtype, kQ, 0, codes, stream);
     return from_cuda(e);
 }
 

@@ -5,8 +5,8 @@
 // ||c||^2 - 2 r.c in float32, a block argmin (lowest index on ties), and for
 // the acoustic levels r -= chosen codeword. It scans all 2048 x 8 codewords,
 // so it is slow (about 4.2 M FMA per frame) but has no candidate pruning.
-// It serves two roles: the re-encode of frames whose tensor-core candidate set
-// could not be certified, and a plain float32 encoder for comparison.
+// It is the plain float32 encoder for comparison; the latency encoder
+// (encode_wide.cu) computes the same scores in the same order.
 #include "handle.cuh"
 
 namespace mimi {
@@ -102,19 +102,6 @@ __global__ void __launch_bounds__(kThreads) k_encode_scan(Tables t, const void* 
         scan_one_frame(t, z, dtype, f, n_q, variant, codes, sz, sy, sr, red_s, red_k);
 }
 
-// Re-encode every frame the tensor-core kernel queued (count read on device).
-__global__ void __launch_bounds__(kThreads) k_rescan(Tables t, const void* z, int dtype, int n_q,
-                                                     int variant, int16_t* codes) {
-    __shared__ float sz[kDin], sy[kD], sr[kD], red_s[kThreads / 32];
-    __shared__ int red_k[kThreads / 32];
-    const int count = min(*t.rescan_count, (int)kRescanCapacity);
-    for (int i = blockIdx.x; i < count; i += gridDim.x)
-        scan_one_frame(t, z, dtype, t.rescan_list[i], n_q, variant, codes, sz, sy, sr, red_s,
-                       red_k);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && count > 0)
-        atomicAdd(&t.stats[1], (unsigned long long)count);
-}
-
 }  // namespace
 
 cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
@@ -122,12 +109,6 @@ cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_
     if (n <= 0) return cudaSuccess;
     const int grid = (int)(n < 148 * 8 ? n : 148 * 8);
     k_encode_scan<<<grid, kThreads, 0, s>>>(t, z, dtype, n, n_q, variant, codes);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_rescan(const Tables& t, const void* z, int dtype, int n_q, int variant,
-                          int16_t* codes, cudaStream_t s) {
-    k_rescan<<<148, kThreads, 0, s>>>(t, z, dtype, n_q, variant, codes);
     return cudaGetLastError();
 }
 

@@ -123,6 +123,11 @@ struct WideArgs {
     float* y;                       // [B][256] projection exchange
     unsigned* bars;                 // [kWideMaxGroups][kWideBarStride] barrier words
     unsigned long long* partial;    // [n_q][groups][FG][S] per-CTA minimum keys
+    // list mode (re-scan of the frames the tensor-core encoder could not certify):
+    // frames list[0 .. min(*list_count, list_cap)), taken B at a time; nullptr: frames 0..B-1
+    const int* list;
+    const int* list_count;
+    int list_cap;
 };
 
 // Copy the codeword rows of chunk c (level c / nch) into buf.
@@ -152,214 +157,235 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
     __shared__ int win_s[FG];
     const int tid = threadIdx.x;
     const int S = a.S;
+    __shared__ int frame_s[FG];
     const int group = blockIdx.x / S, member = blockIdx.x % S;
     const int f0 = group * FG;
-    const int F = min(FG, a.B - f0);
     unsigned* bar = a.bars + group * kWideBarStride;
 
     const int k_lo = member * a.per_k, k_hi = min(kK, k_lo + a.per_k);
     const int nch = (k_hi - k_lo + KS - 1) / KS;
     const int total = a.n_q * nch;
-    issue_chunk<KS>(a, cbuf(0), 0, nch, k_lo, k_hi);
-
-    // ---- y = W_in . z for output dimensions [d0, d1) of every frame of the group,
-    //      each output a sequential FMA chain over j (the full scan's order). The
-    //      latents and W_in rows are staged in passes of JC columns (row stride
-    //      JC + 1: conflict-free column reads), with batched vector loads.
-    {
-        const int per = (kD + S - 1) / S;
-        const int d0 = min(kD, member * per), d1 = min(kD, d0 + per), nd = d1 - d0;
-        const int items = F * nd;
-        const int JC = a.jc, JS = JC + 1, J4 = JC / 4;
-        float* z_s = r_s;             // [F][JS]
-        float* w_s = r_s + F * JS;    // [nd][JS]
-        const int nq_items = (items + kThreads - 1) / kThreads;  // uniform over the CTA
-        int zo[kProjItems], wo[kProjItems];
-        bool act[kProjItems];
-        float acc[kProjItems];
-#pragma unroll
-        for (int q = 0; q < kProjItems; ++q) {
-            const int it = tid + q * kThreads;
-            act[q] = it < items;
-            zo[q] = act[q] ? (it / nd) * JS : 0;
-            wo[q] = act[q] ? (it % nd) * JS : 0;
-            acc[q] = 0.f;
-        }
-        for (int j0 = 0; j0 < kDin; j0 += JC) {
-            __syncthreads();
-            const int nz = F * J4, nt = (F + nd) * J4;
-            for (int e0 = tid; e0 < nt; e0 += 4 * kThreads) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + u * kThreads;
-                    if (e < nz)
-                        v[u] = load_latent4(a.z, a.dtype, (int64_t)(f0 + e / J4) * kDin + j0 + 4 * (e % J4));
-                    else if (e < nt)
-                        v[u] = __ldg(reinterpret_cast<const float4*>(
-                            a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + u * kThreads;
-                    if (e < nt) {
-                        float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
-                        d[0] = v[u].x;
-                        d[1] = v[u].y;
-                        d[2] = v[u].z;
-                        d[3] = v[u].w;
-                    }
-                }
-            }
-            __syncthreads();
-            if (nq_items <= 1) proj_chain<1>(z_s, w_s, zo, wo, acc, JC);
-            else if (nq_items <= 2) proj_chain<2>(z_s, w_s, zo, wo, acc, JC);
-            else if (nq_items <= 4) proj_chain<4>(z_s, w_s, zo, wo, acc, JC);
-            else proj_chain<8>(z_s, w_s, zo, wo, acc, JC);
-        }
-#pragma unroll
-        for (int q = 0; q < kProjItems; ++q)
-            if (act[q]) {
-                const int it = tid + q * kThreads;
-                a.y[(size_t)(f0 + it / nd) * kD + d0 + it % nd] = acc[q];
-            }
-    }
-    unsigned episode = 1;
-    group_arrive(bar);
-    if (!group_wait(bar, S * episode, a.err)) {
-        cp_async_wait_all();
-        return;
-    }
-    for (int e = tid; e < FG * (kD / 4); e += kThreads) {
-        const int f = e / (kD / 4), i4 = e % (kD / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (f < F) v = __ldcg(reinterpret_cast<const float4*>(a.y + (size_t)(f0 + f) * kD) + i4);
-        *reinterpret_cast<float4*>(r_s + f * RSTRIDE + 4 * i4) = v;
-    }
-
     const int tf = tid >> 4, tk = tid & 15;
-    // partial-key reduction: TPF threads per frame (a power of two, <= 32)
-    int tpf = 32;
-    while (tpf * F > kThreads) tpf >>= 1;
-    const int rf = tid / tpf, rsub = tid % tpf;
+    int n_frames = a.B;
+    if (a.list != nullptr) {
+        n_frames = min(__ldcg(a.list_count), a.list_cap);
+        if (blockIdx.x == 0 && tid == 0 && n_frames > 0)
+            atomicAdd(&a.stats[1], (unsigned long long)n_frames);
+    }
+    unsigned episode = 0;
+    int frames_done = 0;
 
-    int c = 0;
-    for (int l = 0; l < a.n_q; ++l) {
-        const float* cn = a.cnorm + (size_t)l * kK;
-        unsigned long long mk[U];
+    for (int base = 0; base < n_frames; base += a.B) {
+        // this group's frames of the batch (all members agree, so a group with none skips it)
+        const int F = min(FG, min(a.B, n_frames - base) - f0);
+        if (F <= 0) continue;
+        const int next_base = base + a.B;
+        const bool final_batch = next_base >= n_frames || n_frames - next_base <= f0;
+        if (tid < F) frame_s[tid] = a.list != nullptr ? __ldg(a.list + base + f0 + tid) : base + f0 + tid;
+        __syncthreads();
+        issue_chunk<KS>(a, cbuf(0), 0, nch, k_lo, k_hi);
+
+        // ---- y = W_in . z for output dimensions [d0, d1) of every frame of the group,
+        //      each output a sequential FMA chain over j (the full scan's order). The
+        //      latents and W_in rows are staged in passes of JC columns (row stride
+        //      JC + 1: conflict-free column reads), with batched vector loads.
+        {
+            const int per = (kD + S - 1) / S;
+            const int d0 = min(kD, member * per), d1 = min(kD, d0 + per), nd = d1 - d0;
+            const int items = F * nd;
+            const int JC = a.jc, JS = JC + 1, J4 = JC / 4;
+            float* z_s = r_s;             // [F][JS]
+            float* w_s = r_s + F * JS;    // [nd][JS]
+            const int nq_items = (items + kThreads - 1) / kThreads;  // uniform over the CTA
+            int zo[kProjItems], wo[kProjItems];
+            bool act[kProjItems];
+            float acc[kProjItems];
 #pragma unroll
-        for (int u = 0; u < U; ++u) mk[u] = ~0ull;
-        for (int kc = k_lo; kc < k_hi; kc += KS, ++c) {
-            const int nk = min(KS, k_hi - kc);
-            cp_async_wait_all();
-            __syncthreads();  // chunk c landed; chunk c - 1 consumed; r_s up to date
-            if (c + 1 < total) issue_chunk<KS>(a, cbuf(c + 1), c + 1, nch, k_lo, k_hi);
-            const float* c_s = cbuf(c);
-            float acc[U][V][4];
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-#pragma unroll
-                for (int v = 0; v < V; ++v)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) acc[u][v][w] = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < kD; i += 4) {
-                float4 rv[U], cv[V];
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    rv[u] = *reinterpret_cast<const float4*>(r_s + (tf + 16 * u) * RSTRIDE + i);
-#pragma unroll
-                for (int v = 0; v < V; ++v)
-                    cv[v] = *reinterpret_cast<const float4*>(c_s + (tk + 16 * v) * RSTRIDE + i);
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        acc[u][v][0] = fmaf(rv[u].x, cv[v].x, acc[u][v][0]);
-                        acc[u][v][1] = fmaf(rv[u].y, cv[v].y, acc[u][v][1]);
-                        acc[u][v][2] = fmaf(rv[u].z, cv[v].z, acc[u][v][2]);
-                        acc[u][v][3] = fmaf(rv[u].w, cv[v].w, acc[u][v][3]);
-                    }
+            for (int q = 0; q < kProjItems; ++q) {
+                const int it = tid + q * kThreads;
+                act[q] = it < items;
+                zo[q] = act[q] ? (it / nd) * JS : 0;
+                wo[q] = act[q] ? (it % nd) * JS : 0;
+                acc[q] = 0.f;
             }
+            for (int j0 = 0; j0 < kDin; j0 += JC) {
+                __syncthreads();
+                const int nz = F * J4, nt = (F + nd) * J4;
+                for (int e0 = tid; e0 < nt; e0 += 4 * kThreads) {
+                    float4 v[4];
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int k = tk + 16 * v;
-                if (k < nk) {
-                    const float cnk = __ldg(cn + kc + k);
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < nz)
+                            v[u] = load_latent4(a.z, a.dtype, (int64_t)frame_s[e / J4] * kDin + j0 + 4 * (e % J4));
+                        else if (e < nt)
+                            v[u] = __ldg(reinterpret_cast<const float4*>(
+                                a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
+                    }
 #pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const float dot = (acc[u][v][0] + acc[u][v][1]) + (acc[u][v][2] + acc[u][v][3]);
-                        mk[u] = umin64(mk[u], pack_key(fmaf(-2.f, dot, cnk), kc + k));
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < nt) {
+                            float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
+                            d[0] = v[u].x;
+                            d[1] = v[u].y;
+                            d[2] = v[u].z;
+                            d[3] = v[u].w;
+                        }
                     }
                 }
+                __syncthreads();
+                if (nq_items <= 1) proj_chain<1>(z_s, w_s, zo, wo, acc, JC);
+                else if (nq_items <= 2) proj_chain<2>(z_s, w_s, zo, wo, acc, JC);
+                else if (nq_items <= 4) proj_chain<4>(z_s, w_s, zo, wo, acc, JC);
+                else proj_chain<8>(z_s, w_s, zo, wo, acc, JC);
             }
-        }
-        // this CTA's minimum per frame -> its slot
-        unsigned long long* part = a.partial + ((size_t)l * a.groups + group) * FG * S;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1)
-                mk[u] = umin64(mk[u], __shfl_xor_sync(0xffffffffu, mk[u], o));
-            const int f = tf + 16 * u;
-            if (tk == 0 && f < F) __stcg(part + (size_t)f * S + member, mk[u]);
+            for (int q = 0; q < kProjItems; ++q)
+                if (act[q]) {
+                    const int it = tid + q * kThreads;
+                    a.y[(size_t)(f0 + it / nd) * kD + d0 + it % nd] = acc[q];
+                }
         }
-        // after the last level only member 0 (which writes the codes) needs the
-        // winners; the others leave once they have arrived
         ++episode;
         group_arrive(bar);
-        const bool last = l == a.n_q - 1;
-        if (last && member != 0) break;
         if (!group_wait(bar, S * episode, a.err)) {
             cp_async_wait_all();
             return;
         }
-        // winners: minimum over the group's S slots of each frame (loads in batches of 4)
-        {
-            unsigned long long m = ~0ull;
-            if (rf < F)
-                for (int s0 = rsub; s0 < S; s0 += 4 * tpf) {
-                    unsigned long long v[4];
+        for (int e = tid; e < FG * (kD / 4); e += kThreads) {
+            const int f = e / (kD / 4), i4 = e % (kD / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (f < F) v = __ldcg(reinterpret_cast<const float4*>(a.y + (size_t)(f0 + f) * kD) + i4);
+            *reinterpret_cast<float4*>(r_s + f * RSTRIDE + 4 * i4) = v;
+        }
+
+        // partial-key reduction: TPF threads per frame (a power of two, <= 32)
+        int tpf = 32;
+        while (tpf * F > kThreads) tpf >>= 1;
+        const int rf = tid / tpf, rsub = tid % tpf;
+
+        int c = 0;
+        for (int l = 0; l < a.n_q; ++l) {
+            const float* cn = a.cnorm + (size_t)l * kK;
+            unsigned long long mk[U];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int sl = s0 + u * tpf;
-                        v[u] = sl < S ? __ldcg(part + (size_t)rf * S + sl) : ~0ull;
-                    }
+            for (int u = 0; u < U; ++u) mk[u] = ~0ull;
+            for (int kc = k_lo; kc < k_hi; kc += KS, ++c) {
+                const int nk = min(KS, k_hi - kc);
+                cp_async_wait_all();
+                __syncthreads();  // chunk c landed; chunk c - 1 consumed; r_s up to date
+                if (c + 1 < total) issue_chunk<KS>(a, cbuf(c + 1), c + 1, nch, k_lo, k_hi);
+                const float* c_s = cbuf(c);
+                float acc[U][V][4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) m = umin64(m, v[u]);
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int v = 0; v < V; ++v)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) acc[u][v][w] = 0.f;
+#pragma unroll 4
+                for (int i = 0; i < kD; i += 4) {
+                    float4 rv[U], cv[V];
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        rv[u] = *reinterpret_cast<const float4*>(r_s + (tf + 16 * u) * RSTRIDE + i);
+#pragma unroll
+                    for (int v = 0; v < V; ++v)
+                        cv[v] = *reinterpret_cast<const float4*>(c_s + (tk + 16 * v) * RSTRIDE + i);
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            acc[u][v][0] = fmaf(rv[u].x, cv[v].x, acc[u][v][0]);
+                            acc[u][v][1] = fmaf(rv[u].y, cv[v].y, acc[u][v][1]);
+                            acc[u][v][2] = fmaf(rv[u].z, cv[v].z, acc[u][v][2]);
+                            acc[u][v][3] = fmaf(rv[u].w, cv[v].w, acc[u][v][3]);
+                        }
                 }
-            for (int o = tpf >> 1; o > 0; o >>= 1) m = umin64(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (rsub == 0 && rf < F) {
-                int w = (int)(uint32_t)m;
-                if (w < 0 || w >= kK) w = 0;  // only reachable with NaN / Inf inputs
-                win_s[rf] = w;
-                if (member == 0) a.codes[(size_t)(f0 + rf) * a.n_q + l] = (int16_t)w;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const int k = tk + 16 * v;
+                    if (k < nk) {
+                        const float cnk = __ldg(cn + kc + k);
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            const float dot = (acc[u][v][0] + acc[u][v][1]) + (acc[u][v][2] + acc[u][v][3]);
+                            mk[u] = umin64(mk[u], pack_key(fmaf(-2.f, dot, cnk), kc + k));
+                        }
+                    }
+                }
+            }
+            // this CTA's minimum per frame -> its slot
+            unsigned long long* part = a.partial + ((size_t)l * a.groups + group) * FG * S;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1)
+                    mk[u] = umin64(mk[u], __shfl_xor_sync(0xffffffffu, mk[u], o));
+                const int f = tf + 16 * u;
+                if (tk == 0 && f < F) __stcg(part + (size_t)f * S + member, mk[u]);
+            }
+            // after the last level only member 0 (which writes the codes) needs the
+            // winners; the others move on once they have arrived
+            ++episode;
+            group_arrive(bar);
+            const bool last = l == a.n_q - 1;
+            if (last && member != 0) break;
+            if (!group_wait(bar, S * episode, a.err)) {
+                cp_async_wait_all();
+                return;
+            }
+            // winners: minimum over the group's S slots of each frame (loads in batches of 4)
+            {
+                unsigned long long m = ~0ull;
+                if (rf < F)
+                    for (int s0 = rsub; s0 < S; s0 += 4 * tpf) {
+                        unsigned long long v[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int sl = s0 + u * tpf;
+                            v[u] = sl < S ? __ldcg(part + (size_t)rf * S + sl) : ~0ull;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) m = umin64(m, v[u]);
+                    }
+                for (int o = tpf >> 1; o > 0; o >>= 1) m = umin64(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (rsub == 0 && rf < F) {
+                    int w = (int)(uint32_t)m;
+                    if (w < 0 || w >= kK) w = 0;  // only reachable with NaN / Inf inputs
+                    win_s[rf] = w;
+                    if (member == 0) a.codes[(size_t)frame_s[rf] * a.n_q + l] = (int16_t)w;
+                }
+            }
+            if (last) {
+                // after the group's last batch every member has arrived for the last
+                // time: reset the count for the next launch (or graph replay)
+                if (final_batch && tid == 0) atomicExch(bar, 0u);
+                break;
+            }
+            __syncthreads();
+            // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
+            if (l < a.n_q - 1 && (l >= 1 || a.variant == 1)) {
+                const float* book = a.C32 + (size_t)l * kK * kD;
+                for (int e = tid; e < F * (kD / 4); e += kThreads) {
+                    const int f = e / (kD / 4), i4 = e % (kD / 4);
+                    const float4 cw = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[f] * kD) + i4);
+                    float4* r = reinterpret_cast<float4*>(r_s + f * RSTRIDE + 4 * i4);
+                    float4 v = *r;
+                    v.x -= cw.x;
+                    v.y -= cw.y;
+                    v.z -= cw.z;
+                    v.w -= cw.w;
+                    *r = v;
+                }
             }
         }
-        if (last) {
-            // every CTA of the group has arrived for the last time: reset the count
-            // for the next launch (or graph replay)
-            if (tid == 0) atomicExch(bar, 0u);
-            break;
-        }
-        __syncthreads();
-        // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
-        if (l < a.n_q - 1 && (l >= 1 || a.variant == 1)) {
-            const float* book = a.C32 + (size_t)l * kK * kD;
-            for (int e = tid; e < F * (kD / 4); e += kThreads) {
-                const int f = e / (kD / 4), i4 = e % (kD / 4);
-                const float4 cw = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[f] * kD) + i4);
-                float4* r = reinterpret_cast<float4*>(r_s + f * RSTRIDE + 4 * i4);
-                float4 v = *r;
-                v.x -= cw.x;
-                v.y -= cw.y;
-                v.z -= cw.z;
-                v.w -= cw.w;
-                *r = v;
-            }
-        }
-    }
-    if (member == 0 && tid == 0) atomicAdd(&a.stats[0], (unsigned long long)F);
+        frames_done += F;
+        __syncthreads();  // frame_s and the buffers are rewritten by the next batch
+    }  // batches
+    if (a.list == nullptr && member == 0 && tid == 0 && frames_done > 0)
+        atomicAdd(&a.stats[0], (unsigned long long)frames_done);
 }
 
 int smem_bytes(int V) { return (2 * 16 * V + FG) * RSTRIDE * 4; }
@@ -435,9 +461,13 @@ cudaError_t encode_wide_configure() {
 }
 
 cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z, int dtype, int B,
-                               int n_q, int variant, int16_t* codes, cudaStream_t s) {
+                               int n_q, int variant, int16_t* codes, cudaStream_t s,
+                               bool rescan_list) {
     if (!p.ok) return cudaErrorInvalidValue;
     WideArgs a;
+    a.list = rescan_list ? t.rescan_list : nullptr;
+    a.list_count = rescan_list ? t.rescan_count : nullptr;
+    a.list_cap = (int)kRescanCapacity;
     a.C32 = t.C32;
     a.Win32 = t.Win32;
     a.cnorm = t.cnorm;

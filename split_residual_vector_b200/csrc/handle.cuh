@@ -13,17 +13,18 @@ constexpr int kD = 256;       // projected width
 constexpr int kK = 2048;      // codewords per codebook
 constexpr int kQ = 8;         // codebooks: 0 semantic, 1..7 acoustic
 
-// Frames whose candidate set could not be certified are re-encoded by the
-// float32 full scan; the work list holds at most this many frames per launch
+// Frames whose candidate set could not be certified are re-encoded in float32
+// by the wide encoder; the work list holds at most this many frames per launch
 // of the tensor-core kernel (encode is split into chunks of this size, so the
 // list cannot overflow).
 constexpr int64_t kRescanCapacity = 1 << 20;
 
 // Largest streaming step the latency (wide) encoder takes; larger steps go to
-// the tensor-core encoder, which is as fast from about 900 frames up (measured
-// per-call latency on B200: 54 us at 1 frame, 121 us at 128, 318 us at 768,
-// 392 us at 1024, against 290-380 us for the tensor-core encoder).
-constexpr int kWideMaxFrames = 896;
+// the tensor-core encoder. Measured per-call latency on B200: 54 us at 1 frame,
+// 121 us at 128, 318 us at 768, 392 us at 1024; the tensor-core encoder takes
+// 290-380 us plus, from a few hundred frames up, the float32 re-scan of its
+// (usually one or two) uncertified frames, ~400 us for a single frame.
+constexpr int kWideMaxFrames = 1024;
 constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
 constexpr int kWideMaxGroups = 64;    // group barriers
 constexpr int kWideBarStride = 32;    // words per group barrier (count, generation; own 128 B line)
@@ -67,8 +68,6 @@ cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t 
 // encode_scan.cu
 cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                                int variant, int16_t* codes, cudaStream_t s);
-cudaError_t launch_rescan(const Tables& t, const void* z, int dtype, int n_q, int variant,
-                          int16_t* codes, cudaStream_t s);
 // encode_wide.cu
 struct WidePlan {
     bool ok = false;   // false: B is outside (0, kWideMaxFrames] or needs more CTAs than SMs
@@ -84,8 +83,11 @@ WidePlan plan_encode_wide(int B, int num_sms);
 size_t wide_partial_bytes(int num_sms);
 cudaError_t encode_wide_configure();  // once per device, before the first launch
 // Launches on one set of tables must be stream-ordered (they share the scratch).
+// rescan_list: encode the frames of t.rescan_list (count on the device), B at a
+// time with plan p, instead of frames 0..B-1.
 cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z, int dtype, int B,
-                               int n_q, int variant, int16_t* codes, cudaStream_t s);
+                               int n_q, int variant, int16_t* codes, cudaStream_t s,
+                               bool rescan_list = false);
 // decode.cu
 cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int n_q, float* out,
                           cudaStream_t s);

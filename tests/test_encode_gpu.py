@@ -133,11 +133,11 @@ def test_streaming_step_equals_full_scan(dtype):
     """Small steps run the latency encoder, whose scores are the float32 full scan's
     (same sums in the same order): every code equals encode_scan's, near ties included.
     Sizes span one to 64 frame groups, ragged group tails and every thread-tile shape."""
-    model, frames = synth.streaming_step(896, calls=1)
+    model, frames = synth.streaming_step(1024, calls=1)
     q = quantizer(model)
     z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
     zd = to_device(np.ascontiguousarray(z))
-    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 833, 896)
+    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 896, 1000, 1024)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         scan = q.encode_scan(zd[:b]).cpu().numpy()
@@ -147,9 +147,9 @@ def test_streaming_step_equals_full_scan(dtype):
     assert q.get_error() == 0
 
 
-@pytest.mark.parametrize("batch", [897, 1024, 5000])
+@pytest.mark.parametrize("batch", [1025, 5000])
 def test_streaming_step_large_batch_uses_the_batch_encoder(batch):
-    """Above the latency encoder's batch limit (896) a step is a batch encode."""
+    """Above the latency encoder's batch limit (1024) a step is a batch encode."""
     model, frames = synth.streaming_step(batch, calls=1)
     q = quantizer(model)
     codes = q.encode_step(to_device(np.ascontiguousarray(frames[0]))).cpu().numpy()
@@ -224,6 +224,26 @@ def test_many_equal_codewords_go_to_the_full_scan():
     assert (codes[:, 0] == tied[0]).all()
     _, rescanned = q.stats()
     assert rescanned == 3
+
+
+def test_rescan_of_many_frames_in_several_batches():
+    """Every level-1 codeword has ~20 exact copies, so no frame's candidate window can be
+    certified and all 2500 frames are re-encoded by the float32 wide encoder, 1024 at a time
+    (three batches). Its scores are the full scan's, so the codes equal encode_scan's; they
+    also match the oracle (ties between copies go to the lowest index on both sides)."""
+    model = _small_model(seed=33)
+    model.C[1] = model.C[1][np.arange(2048) % 100]
+    q = quantizer(model)
+    rng = np.random.default_rng(34)
+    z = rng.standard_normal((2500, 512)).astype(np.float32)
+    zd = to_device(z)
+    codes = q.encode(zd).cpu().numpy()
+    enc, rescanned = q.stats()
+    assert enc == 2500 and rescanned == 2500
+    assert np.array_equal(codes, q.encode_scan(zd).cpu().numpy())
+    ref, db, ds = oracle.encode(z, model.W_in, model.C)
+    assert_codes_match(codes, ref, db, ds, "all frames re-scanned")
+    assert q.get_error() == 0
 
 
 def test_zero_huge_and_tiny_latents():
