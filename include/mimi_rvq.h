@@ -175,6 +175,18 @@ int mimi_rvq_decode_ex(mimi_rvq_t h, const int16_t *codes, int64_t N, int n_q, f
 int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st *stream);
 
 /*
+ * Self-test of the failure path: launches one small kernel on `stream` whose
+ * wait can never complete -- which = 0: an mbarrier phase nothing completes
+ * (the tensor-core encoder's kind of wait); which = 1: a group barrier that
+ * only one of its two members reaches (the wide encoder's kind of wait). The
+ * kernel gives up after about 50 ms, records the timeout and returns, so the
+ * next mimi_rvq_get_error returns MIMI_RVQ_ETIMEOUT (and resets the state a
+ * timeout can leave behind); the handle stays usable. Returns MIMI_RVQ_EINVAL
+ * for another `which`.
+ */
+int mimi_rvq_wait_selftest(mimi_rvq_t h, int which, struct CUstream_st *stream);
+
+/*
  * Counters since create (synchronises `stream`): frames encoded, and frames
  * whose bf16 candidate pass could not certify its candidate set at some level
  * and were re-encoded by the full float32 scan. Either pointer may be NULL.

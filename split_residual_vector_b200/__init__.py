@@ -23,7 +23,7 @@ EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_e
            "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
            "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror",
            "mimi_rvq_encode_profile", "mimi_rvq_delay_pack", "mimi_rvq_delay_unpack",
-           "mimi_rvq_embed_sum")
+           "mimi_rvq_embed_sum", "mimi_rvq_wait_selftest")
 TEXT_CARD, TEXT_PAD, AUDIO_PAD = 32000, 32000, 2048
 
 _lib = None
@@ -70,6 +70,8 @@ def library() -> ctypes.CDLL:
     lib.mimi_rvq_stats.restype = ci
     lib.mimi_rvq_strerror.argtypes = [ci]
     lib.mimi_rvq_strerror.restype = ctypes.c_char_p
+    lib.mimi_rvq_wait_selftest.argtypes = [vp, ci, vp]
+    lib.mimi_rvq_wait_selftest.restype = ci
     i32 = ctypes.c_int32
     lib.mimi_rvq_delay_pack.argtypes = [vp, vp, ci, i64, vp, i64, i32, i32, vp, vp]
     lib.mimi_rvq_delay_pack.restype = ci
@@ -221,6 +223,12 @@ class Quantizer:
                "mimi_rvq_encode_profile")
         vals = cyc.cpu().tolist()
         return out, dict(zip(self.PROFILE_SLOTS, vals))
+
+    def wait_selftest(self, which: int, stream=None):
+        """Launch a kernel whose wait never completes (0: mbarrier, 1: group barrier); it
+        times out after ~50 ms. The next get_error() returns -6 (timed out)."""
+        _check(library().mimi_rvq_wait_selftest(self._h, int(which), _stream(stream)),
+               "mimi_rvq_wait_selftest")
 
     def get_error(self, stream=None) -> int:
         """Synchronise the stream; return and clear the device error status (0 = ok)."""

@@ -291,6 +291,13 @@ int mimi_rvq_decode(mimi_rvq_t h, const int16_t* codes, int64_t N, float* latent
     return mimi_rvq_decode_ex(h, codes, N, kQ, latents, stream);
 }
 
+int mimi_rvq_wait_selftest(mimi_rvq_t h, int which, struct CUstream_st* stream) {
+    if (!h || (which != 0 && which != 1)) return MIMI_RVQ_EINVAL;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MIMI_RVQ_EINVAL;
+    return from_cuda(mimi::launch_wait_selftest(h->t, which, stream));
+}
+
 int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st* stream) {
     if (!h) return MIMI_RVQ_EINVAL;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MIMI_RVQ_ECUDA;

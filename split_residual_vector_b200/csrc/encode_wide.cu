@@ -66,37 +66,6 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Barrier among the S CTAs of one group: bar[0] counts arrivals and reaches
-// S * e when episode e is complete. arrive() adds this CTA's arrival (after
-// its writes); wait() spins (bounded) until the count reaches the target.
-// Returns false (and records a timeout) if the wait runs out.
-__device__ __forceinline__ void group_arrive(unsigned* bar) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
-    }
-}
-
-__device__ bool group_wait(unsigned* bar, unsigned target, int* err) {
-    int ok = 1;
-    if (threadIdx.x == 0) {
-        const long long t0 = clock64();
-        while (true) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-            if (v >= target) break;
-            if (clock64() - t0 > kWaitBudgetCycles) {
-                atomicOr(err, MIMI_DEV_ERR_TIMEOUT);
-                ok = 0;
-                break;
-            }
-        }
-        __threadfence();
-    }
-    return __syncthreads_and(ok) != 0;
-}
-
 // y = W_in . z outputs of this thread: NQ items (tid + q * 256) with offsets
 // zo / wo into the staged latents and W_in rows, each a sequential FMA chain
 // over the JC staged columns (inactive items compute on clamped offsets and

@@ -26,7 +26,7 @@ constexpr int64_t kRescanCapacity = 1 << 20;
 // (usually one or two) uncertified frames, ~400 us for a single frame.
 constexpr int kWideMaxFrames = 1024;
 constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
-constexpr int kWideMaxGroups = 64;    // group barriers
+constexpr int kWideMaxGroups = 64;    // group barriers (the last one is the wait self-test's)
 constexpr int kWideBarStride = 32;    // words per group barrier (count, generation; own 128 B line)
 
 struct Tables {
@@ -88,6 +88,10 @@ cudaError_t encode_wide_configure();  // once per device, before the first launc
 cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z, int dtype, int B,
                                int n_q, int variant, int16_t* codes, cudaStream_t s,
                                bool rescan_list = false);
+// selftest.cu: a kernel whose wait can never complete (which 0: an mbarrier,
+// as the tensor-core encoder waits; 1: a group barrier, as the wide encoder
+// waits); it times out after ~50 ms and records MIMI_DEV_ERR_TIMEOUT.
+cudaError_t launch_wait_selftest(const Tables& t, int which, cudaStream_t s);
 // decode.cu
 cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int n_q, float* out,
                           cudaStream_t s);

@@ -58,18 +58,52 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // records a timeout) if the budget runs out or another thread of the CTA has
 // already given up (*abort != 0).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
+                                          int* err, long long budget = kWaitBudgetCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitBudgetCycles) {
+        if (clock64() - t0 > budget) {
             *abort = 1;
             atomicOr(err, MIMI_DEV_ERR_TIMEOUT);
             return false;
         }
     }
+}
+
+// ------------------------------------------------------------------ grid-level group barrier
+
+// Barrier among the CTAs of one group of a cooperative launch: *bar counts
+// arrivals and reaches S * e when episode e is complete. group_arrive adds this
+// CTA's arrival (after its writes); group_wait spins (bounded) until the count
+// reaches the target and returns false (recording a timeout) if it runs out.
+__device__ __forceinline__ void group_arrive(unsigned* bar) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+    }
+}
+
+__device__ __forceinline__ bool group_wait(unsigned* bar, unsigned target, int* err,
+                                           long long budget = kWaitBudgetCycles) {
+    int ok = 1;
+    if (threadIdx.x == 0) {
+        const long long t0 = clock64();
+        while (true) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= target) break;
+            if (clock64() - t0 > budget) {
+                atomicOr(err, MIMI_DEV_ERR_TIMEOUT);
+                ok = 0;
+                break;
+            }
+        }
+        __threadfence();
+    }
+    return __syncthreads_and(ok) != 0;
 }
 
 // ------------------------------------------------------------------ TMA
