@@ -54,7 +54,9 @@ MOSHI_DELAYS = [0, 1, 1, 1, 1, 1, 1, 1]   # acoustic delay 1 (the final model's)
 # DRAM bytes (read + write) per unit from one ncu capture of the current kernel, with the
 # summary that records it; the bench scales it by the units of a launch. None: not captured.
 NCU_TRAFFIC_PER_UNIT = {
-    "k_embed_sum": (48_951, "profiles/k_embed_sum_moshi_input.md"),   # per step
+    "k_embed_sum": (48_951, "profiles/k_embed_sum_moshi_input.md"),        # per step
+    "k_encode_tc/f32": (2_467, "profiles/k_encode_tc_offline_batch.md"),   # per fp32 frame
+    "k_decode": (1_990, "profiles/k_decode_decode_heavy.md"),              # per frame
 }
 
 
@@ -333,21 +335,27 @@ def run_ours(args, rank, world, local_rank):
     lat_bytes = 2048 if work.get("dtype", "f32") == "f32" else 1024
     if do_enc:
         tf = ENC_FLOP * n / (enc_avg / 1e3) / 1e12
+        tr = NCU_TRAFFIC_PER_UNIT["k_encode_tc/f32"] if work.get("dtype", "f32") == "f32" else None
         kernels.append({
-            "kernel": "encode call (k_encode_tc + full-scan fallback)", "bound": "tensor",
+            "kernel": "encode call (k_encode_tc + float32 re-encode)", "bound": "tensor",
             "achieved": tf, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-            "frac": tf / peaks["bf16_tflops_sustained"], "traffic": None, "ms": enc_avg,
+            "frac": tf / peaks["bf16_tflops_sustained"],
+            "traffic": tr[0] * n if tr else None, "traffic_source": tr[1] if tr else None,
+            "ms": enc_avg,
             "algorithmic": f"{ENC_FLOP} FLOP/frame x {n} frames; HBM {lat_bytes + 16} B/frame",
             "hbm_gbs": (lat_bytes + 16) * n / (enc_avg / 1e3) / 1e9})
     if do_dec:
         gbs = DEC_BYTES * n / (dec_avg / 1e3) / 1e9
+        tr = NCU_TRAFFIC_PER_UNIT["k_decode"]
         kernels.append({
             "kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None, "ms": dec_avg,
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": tr[0] * n,
+            "traffic_source": tr[1], "ms": dec_avg,
             "algorithmic": f"{DEC_BYTES} B/frame x {n} frames (codes in, fp32 latents out)"})
     dominant = kernels[0]
     roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = dominant["kernel"]
+    roofline["traffic_source"] = dominant.get("traffic_source")
     roofline["peak_source"] = (f"{peaks['source']} "
                                f"{'bf16_tflops_sustained' if dominant['bound'] == 'tensor' else 'hbm_gbs'}")
     if args.self_profile and do_enc:
