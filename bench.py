@@ -151,6 +151,35 @@ class ClockSampler:
                 "samples": len(load)}
 
 
+# --------------------------------------------------------------------- ranks
+
+
+def init_dist(world, backend="nccl"):
+    """One process per GPU: the process group for world > 1 (None for one rank). A short
+    timeout makes ranks that wait on one another end with an error."""
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x, dist, device):
+    """The largest value of x over all ranks (x itself with one rank)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Units per second of the whole job: every rank processes units_per_rank per step (weak
+    scaling) and the step time is the slowest rank's."""
+    return units_per_rank * world / (ms_per_step / 1e3)
+
+
 # --------------------------------------------------------------------- workloads
 
 
@@ -212,10 +241,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist(world)
 
     name = args.workload
     work = make_workload(name, rank, args.frames)
@@ -269,16 +295,12 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
-    elapsed_ms = start.elapsed_time(stop)
-    if dist:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist, device)
     status = q.get_error(stream)
     enc_avg = sum(a.elapsed_time(b) for a, b in enc_ms) / max(len(enc_ms), 1)
     dec_avg = sum(a.elapsed_time(b) for a, b in dec_ms) / max(len(dec_ms), 1)
     ms_per_step = elapsed_ms / args.steps
-    value = n * world / (ms_per_step / 1e3)
+    value = whole_job_rate(n, world, ms_per_step)
 
     # ---- end to end through the public API, host buffers (pinned), copies inside
     e2e = None
@@ -317,12 +339,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = a.elapsed_time(b) / k
-        if dist:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": n * world / (e_ms / 1e3), "unit": "frames/s", "h2d_bytes_per_step": bi,
+        e_ms = max_over_ranks(a.elapsed_time(b) / k, dist, device)
+        e2e = {"value": whole_job_rate(n, world, e_ms), "unit": "frames/s", "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e_ms, "steps": k}
 
     if rank != 0:
@@ -433,10 +451,7 @@ def run_moshi_input(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist(world)
     T = args.frames or (1 << 16)
     text_h, audio_h = synth.moshi_streams(T, seed=5 + 100 * rank)
     rows = synth.moshi_rows()
@@ -481,13 +496,9 @@ def run_moshi_input(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
-    elapsed_ms = start.elapsed_time(stop)
-    if dist:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist, device)
     ms_per_step = elapsed_ms / args.steps
-    value = T * world / (ms_per_step / 1e3)
+    value = whole_job_rate(T, world, ms_per_step)
     pack_avg = sum(a.elapsed_time(b) for a, b in pack_ms) / len(pack_ms)
     emb_avg = sum(a.elapsed_time(b) for a, b in emb_ms) / len(emb_ms)
     bad = int(n_bad.item())
@@ -518,12 +529,8 @@ def run_moshi_input(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = a.elapsed_time(b) / k
-        if dist:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": T * world / (e_ms / 1e3), "unit": "frames/s",
+        e_ms = max_over_ranks(a.elapsed_time(b) / k, dist, device)
+        e2e = {"value": whole_job_rate(T, world, e_ms), "unit": "frames/s",
                "h2d_bytes_per_step": text.numel() * 4 + audio.numel() * 2,
                "d2h_bytes_per_step": out.numel() * 2, "ms_per_step": e_ms, "steps": k}
     if rank != 0:

@@ -1,0 +1,62 @@
+"""The multi-rank host logic of the benchmark, on CPU with the gloo backend and two ranks:
+every rank gets its own workload (weak scaling), the step time is the slowest rank's, the
+whole-job rate counts every rank's units, and the reference arm runs on rank 0 alone."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch
+    import bench
+    dist = bench.init_dist(world, backend="gloo")
+    slowest = bench.max_over_ranks(1.5 * (rank + 1), dist, "cpu")
+    work = bench.make_workload("offline_batch", rank, frames=4)
+    row = torch.from_numpy(work["z"][0, :8].copy())
+    rows = [torch.empty_like(row) for _ in range(world)]
+    dist.all_gather(rows, row)
+    rate = bench.whole_job_rate(work["frames"], world, slowest)
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, slowest, [r.tolist() for r in rows], rate))
+
+
+def test_two_gloo_ranks():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(out.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, slowest, rows, rate in results:
+        assert slowest == 3.0                      # the max over ranks, on every rank
+        assert rows[0] != rows[1]                  # each rank drew its own workload
+        assert rate == pytest.approx(4 * 2 / 3.0e-3)
+    assert results[0][2] == results[1][2]          # both ranks saw the same gathered rows
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
