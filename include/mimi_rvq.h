@@ -110,6 +110,13 @@ int mimi_rvq_encode_step(mimi_rvq_t h, const void *frames, int dtype, int B,
                          int16_t *codes, struct CUstream_st *stream);
 
 /*
+ * Streaming step with options: n_q and variant as for mimi_rvq_encode_ex
+ * (codes [B][n_q]); otherwise as mimi_rvq_encode_step.
+ */
+int mimi_rvq_encode_step_ex(mimi_rvq_t h, const void *frames, int dtype, int B, int n_q,
+                            int variant, int16_t *codes, struct CUstream_st *stream);
+
+/*
  * Encode with options. n_q in 1..8 keeps only the first n_q codebooks (the
  * semantic one and n_q - 1 acoustic levels: quantizer dropout at inference,
  * for a lower bit-rate); codes are then [N][n_q]. variant 0 is the split RVQ

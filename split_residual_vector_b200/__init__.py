@@ -23,7 +23,7 @@ EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_e
            "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
            "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror",
            "mimi_rvq_encode_profile", "mimi_rvq_delay_pack", "mimi_rvq_delay_unpack",
-           "mimi_rvq_embed_sum", "mimi_rvq_wait_selftest")
+           "mimi_rvq_embed_sum", "mimi_rvq_wait_selftest", "mimi_rvq_encode_step_ex")
 TEXT_CARD, TEXT_PAD, AUDIO_PAD = 32000, 32000, 2048
 
 _lib = None
@@ -70,6 +70,8 @@ def library() -> ctypes.CDLL:
     lib.mimi_rvq_stats.restype = ci
     lib.mimi_rvq_strerror.argtypes = [ci]
     lib.mimi_rvq_strerror.restype = ctypes.c_char_p
+    lib.mimi_rvq_encode_step_ex.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
+    lib.mimi_rvq_encode_step_ex.restype = ci
     lib.mimi_rvq_wait_selftest.argtypes = [vp, ci, vp]
     lib.mimi_rvq_wait_selftest.restype = ci
     i32 = ctypes.c_int32
@@ -161,12 +163,17 @@ class Quantizer:
         _check(st, "mimi_rvq_encode")
         return out
 
-    def encode_step(self, frames, out=None, stream=None):
-        """frames [B, 512] (one frame per stream) -> codes [B, 8] int16."""
+    def encode_step(self, frames, out=None, stream=None, n_q=NUM_CODEBOOKS, variant=0):
+        """frames [B, 512] (one frame per stream) -> codes [B, n_q] int16."""
         b, dt = self._latents(frames)
-        out = self._codes_out(b, out)
-        _check(library().mimi_rvq_encode_step(self._h, frames.data_ptr(), dt, b, out.data_ptr(),
-                                              _stream(stream)), "mimi_rvq_encode_step")
+        out = self._codes_out(b, out, n_q)
+        if n_q == NUM_CODEBOOKS and variant == 0:
+            st = library().mimi_rvq_encode_step(self._h, frames.data_ptr(), dt, b, out.data_ptr(),
+                                                _stream(stream))
+        else:
+            st = library().mimi_rvq_encode_step_ex(self._h, frames.data_ptr(), dt, b, n_q, variant,
+                                                   out.data_ptr(), _stream(stream))
+        _check(st, "mimi_rvq_encode_step")
         return out
 
     def project(self, latents, out=None, stream=None):

@@ -232,17 +232,22 @@ int mimi_rvq_encode(mimi_rvq_t h, const void* latents, int dtype, int64_t N, int
     return mimi_rvq_encode_ex(h, latents, dtype, N, kQ, 0, codes, stream);
 }
 
-int mimi_rvq_encode_step(mimi_rvq_t h, const void* frames, int dtype, int B, int16_t* codes,
-                         struct CUstream_st* stream) {
-    if (B < 0) return MIMI_RVQ_EINVAL;
-    if (!h) return MIMI_RVQ_EINVAL;
-    const mimi::WidePlan p = mimi::plan_encode_wide(B, h->num_sms);
-    if (!p.ok) return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, kQ, 0, codes, stream);
+int mimi_rvq_encode_step_ex(mimi_rvq_t h, const void* frames, int dtype, int B, int n_q,
+                            int variant, int16_t* codes, struct CUstream_st* stream) {
+    if (!h || B < 0) return MIMI_RVQ_EINVAL;
     if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
+    if (n_q < 1 || n_q > kQ || (variant != 0 && variant != 1)) return MIMI_RVQ_EINVAL;
+    const mimi::WidePlan p = mimi::plan_encode_wide(B, h->num_sms);
+    if (!p.ok) return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, n_q, variant, codes, stream);
     const int c = check_common(h, frames, codes, B);
     if (c <= 0) return c;
     return from_cuda(
-        mimi::launch_encode_wide(h->t, p, frames, dtype, B, kQ, 0, codes, stream));
+        mimi::launch_encode_wide(h->t, p, frames, dtype, B, n_q, variant, codes, stream));
+}
+
+int mimi_rvq_encode_step(mimi_rvq_t h, const void* frames, int dtype, int B, int16_t* codes,
+                         struct CUstream_st* stream) {
+    return mimi_rvq_encode_step_ex(h, frames, dtype, B, kQ, 0, codes, stream);
 }
 
 int mimi_rvq_encode_profile(mimi_rvq_t h, const void* latents, int dtype, int64_t N,

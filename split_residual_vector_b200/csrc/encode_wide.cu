@@ -69,14 +69,27 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // y = W_in . z outputs of this thread: NQ items (tid + q * 256) with offsets
 // zo / wo into the staged latents and W_in rows, each a sequential FMA chain
 // over the JC staged columns (inactive items compute on clamped offsets and
-// are never stored).
+// are never stored). Operands are read into registers JB columns at a time
+// before the chain steps that use them, so shared-memory latency is paid once
+// per batch rather than once per step.
 template <int NQ>
 __device__ __forceinline__ void proj_chain(const float* z_s, const float* w_s, const int* zo,
                                            const int* wo, float* acc, int JC) {
-#pragma unroll 8
-    for (int j = 0; j < JC; ++j)
+    constexpr int JB = NQ >= 8 ? 4 : (NQ >= 4 ? 8 : 16);  // divides JC (a multiple of 16)
+    for (int j0 = 0; j0 < JC; j0 += JB) {
+        float wv[NQ][JB], zv[NQ][JB];
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) acc[q] = fmaf(w_s[wo[q] + j], z_s[zo[q] + j], acc[q]);
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+            for (int j = 0; j < JB; ++j) {
+                wv[q][j] = w_s[wo[q] + j0 + j];
+                zv[q][j] = z_s[zo[q] + j0 + j];
+            }
+#pragma unroll
+        for (int j = 0; j < JB; ++j)
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) acc[q] = fmaf(wv[q][j], zv[q][j], acc[q]);
+    }
 }
 
 struct WideArgs {

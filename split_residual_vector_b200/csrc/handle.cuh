@@ -80,6 +80,7 @@ struct WidePlan {
     int smem = 0;      // dynamic shared memory bytes
 };
 WidePlan plan_encode_wide(int B, int num_sms);
+
 size_t wide_partial_bytes(int num_sms);
 cudaError_t encode_wide_configure();  // once per device, before the first launch
 // Launches on one set of tables must be stream-ordered (they share the scratch).

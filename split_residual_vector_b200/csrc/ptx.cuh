@@ -241,11 +241,6 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
     return r;
 }
 
-// Barrier over a subset of the block's warps (id 1..15, count a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

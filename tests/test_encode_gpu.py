@@ -130,9 +130,9 @@ def test_streaming_step(batch):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_streaming_step_equals_full_scan(dtype):
-    """Small steps run the latency encoder, whose scores are the float32 full scan's
-    (same sums in the same order): every code equals encode_scan's, near ties included.
-    Sizes span one to 64 frame groups, ragged group tails and every thread-tile shape."""
+    """Small steps run the latency encoder, whose scores are the float32 full scan's (same
+    sums in the same order): every code equals encode_scan's, near ties included. Sizes span
+    one to 16 frame groups, ragged group tails and every thread-tile shape."""
     model, frames = synth.streaming_step(1024, calls=1)
     q = quantizer(model)
     z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
@@ -144,6 +144,17 @@ def test_streaming_step_equals_full_scan(dtype):
         assert np.array_equal(step, scan), f"B={b}: {np.argwhere(step != scan)[:5]}"
     enc, _ = q.stats()
     assert enc == sum(sizes)
+    assert q.get_error() == 0
+
+
+def test_streaming_step_fewer_codebooks_and_variant():
+    model, frames = synth.streaming_step(300, calls=1)
+    q = quantizer(model)
+    zd = to_device(np.ascontiguousarray(frames[0]))
+    for n_q, variant in ((1, 0), (5, 0), (8, 1), (3, 1)):
+        step = q.encode_step(zd, n_q=n_q, variant=variant).cpu().numpy()
+        scan = q.encode_scan(zd, n_q=n_q, variant=variant).cpu().numpy()
+        assert step.shape == (300, n_q) and np.array_equal(step, scan), (n_q, variant)
     assert q.get_error() == 0
 
 

@@ -26,7 +26,7 @@ def test_a_wait_that_never_completes_times_out_and_the_handle_recovers(which):
     q.wait_selftest(which)
     assert q.get_error() == ETIMEOUT          # reported once ...
     assert q.get_error() == 0                 # ... and cleared
-    # both encoders (the wide one uses the group barriers the timeout may have left
+    # both encoders (the streaming one uses the group barriers the timeout may have left
     # mid-count) still give the same codes
     assert np.array_equal(q.encode_step(z).cpu().numpy(), before)
     assert np.array_equal(q.encode(z).cpu().numpy(), before_tc)
