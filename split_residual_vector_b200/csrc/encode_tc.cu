@@ -12,7 +12,8 @@
 //      candidate scores ||c||^2 - 2 bf16(r) . bf16(c) for all 2048 codewords
 //      as 16 tcgen05 GEMM tiles [128 x 256] x [256 x 128] (codebook tiles
 //      streamed by TMA into a shared-memory ring; accumulators double-buffered
-//      in TMEM columns [256, 512)). The epilogue keeps a sorted top-8 per row.
+//      in TMEM columns [256, 512)). The epilogue keeps a sorted list of the
+//      best 8 candidate keys per row.
 //   3. certified pick: with E a rigorous bound on |bf16 score - exact score|
 //      (from ||r||, this row's bf16 rounding residual ||bf16(r) - r||, and the
 //      codebook's max ||c|| and max ||bf16(c) - c||), every codeword outside
@@ -20,15 +21,17 @@
 //      s_8 > s_1 + 2E; the candidates within s_1 + 2E are re-scored in float32
 //      (||c||^2 - 2 r.c with r read from TMEM and c from the float32
 //      codebook); a single candidate needs no re-score. If the top-8 cannot be
-//      certified the frame is queued for the float32 full scan.
+//      certified the frame is queued for a float32 re-encode (the wide encoder,
+//      in list mode, after this kernel).
 //   4. acoustic levels: r -= c_win in TMEM, and bf16(r) is written into the
 //      shared-memory A operand of the next level.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues the MMAs (one thread), warps 2..5 are the epilogue (thread = frame row
-// = TMEM lane). The semantic level (0) and acoustic level 1 share the A
-// operand bf16(y), so the tensor core runs from level 0 into level 1 while the
-// epilogue re-scores level 0.
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
+// issues the MMAs (one thread), warps 2..9 are the epilogue: the two warps of a
+// TMEM lane quarter (frame rows 32q .. 32q + 31) split each score tile's
+// columns and the residual's dimensions between them. The semantic level (0)
+// and acoustic level 1 share the A operand bf16(y), so the tensor core runs
+// from level 0 into level 1 while the epilogue re-scores level 0.
 #include <cuda.h>
 
 #include "handle.cuh"
