@@ -207,29 +207,33 @@ def to_device_latents(torch, z, dtype, device):
 
 
 def cpu_baseline(work, name, budget_s=12.0):
-    """The float64 oracle on this host's cores over a bounded sample of the workload."""
+    """The float64 oracle on this host's cores over a bounded sample of the workload, and the
+    same on one thread over a small slice."""
     import oracle
     m = work["model"]
     cores = oracle.threads(0)
 
-    def run(n):
+    def run(n, nthreads=0):
         t0 = time.perf_counter()
         if name in ("offline_batch", "bulk_tokenization"):
-            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C)
+            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C, nthreads=nthreads)
             if name == "offline_batch":
-                oracle.decode(codes, m.C, m.W_out)
+                oracle.decode(codes, m.C, m.W_out, nthreads=nthreads)
         else:
-            oracle.decode(work["codes"][:n], m.C, m.W_out)
+            oracle.decode(work["codes"][:n], m.C, m.W_out, nthreads=nthreads)
         return time.perf_counter() - t0
 
     n = 64 if name != "decode_heavy" else 4096
     dt = run(n)
     n = int(max(n, min(work["frames"], n * budget_s / max(dt, 1e-3))))
     dt = run(n)
+    n1 = 32 if name != "decode_heavy" else 4096
+    dt1 = run(n1, nthreads=1)
     what = {"offline_batch": "encode+decode", "bulk_tokenization": "encode",
             "decode_heavy": "decode"}[name]
     return {"value": n / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n} frames of the workload, {what}, float64 oracle, {dt:.1f} s"}
+            "sample": f"first {n} frames of the workload, {what}, float64 oracle, {dt:.1f} s",
+            "one_thread": {"value": n1 / dt1, "unit": "frames/s", "sample": f"first {n1} frames"}}
 
 
 # --------------------------------------------------------------------- our arm
