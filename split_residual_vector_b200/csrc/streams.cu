@@ -6,11 +6,16 @@
 // Packing and unpacking are index shifts: one thread per output token, the
 // delays passed by value. The embedding sum is a gather bound by memory: for
 // each step, K table rows of d elements are read (K = 17, d = 4096: 139 KB in
-// bf16) and one row of d is written. bf16 tables with K <= 28 take the
-// pipelined kernel (cp.async copies of several stages in flight, below);
-// otherwise one CTA per step, each thread issuing the loads of up to 8 tables'
-// rows before adding them. The sum is float32, table k in order; the output is
-// stored with evict-first hints so the hot table rows keep the L2.
+// bf16) and one row of d is written. Three forms, chosen by shape:
+//   - bf16 tables of d = 4096 (the Temporal Transformer's width), K <= 32: a
+//     producer/consumer kernel that copies whole table rows into a shared-
+//     memory ring with bulk copies (k_embed_sum_tma);
+//   - other bf16 shapes with K <= 28: each thread copies its own 16-byte
+//     pieces of several stages ahead with cp.async (k_embed_sum_async);
+//   - otherwise (float32 tables, more tables): one CTA per step, each thread
+//     issuing the loads of up to 8 tables' rows before adding them.
+// The sum is float32, table k in order; outputs are stored with evict-first
+// hints so the hot table rows keep the L2.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -313,16 +318,6 @@ __device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t x) {
         "add.rn.f32.bf16 %1, hi, %1;\n\t}"
         : "+f"(a), "+f"(b)
         : "r"(x));
-}
-
-__device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
-}
-__device__ __forceinline__ void store4(__nv_bfloat16* p, const float (&v)[4]) {
-    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-    const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-    __stcs(reinterpret_cast<uint2*>(p),
-           make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b)));
 }
 
 template <int NST, typename OT, int D>
