@@ -117,6 +117,26 @@ def test_bulk_tokenization_bf16_full_size_sampled():
     print("bulk sampled", assert_codes_match(codes[idx], ref, db, ds, "bulk_tokenization"))
 
 
+@pytest.mark.parametrize("workload", ["offline_batch", "bulk_tokenization"])
+def test_every_frame_of_the_full_size_workloads(workload):
+    """Every frame of the 240 000- and 1 048 576-frame encodes: the tensor-core codes are
+    compared with the float32 full scan's on the GPU, and every frame where the two differ goes
+    to the float64 oracle, which must find a near-tie there (the only frames where two correct
+    float32 encoders may disagree)."""
+    work = getattr(synth, workload)()
+    q = quantizer(work.model)
+    z = to_device(work.z)
+    tc = q.encode(z).cpu().numpy()
+    scan = q.encode_scan(z).cpu().numpy()
+    assert q.get_error() == 0
+    diff = np.nonzero(np.any(tc != scan, axis=1))[0]
+    print(workload, "frames where the encoders differ:", len(diff), "of", len(tc))
+    assert len(diff) < 0.05 * len(tc)
+    if len(diff):
+        _, db, ds = oracle.encode(work.z[diff], work.model.W_in, work.model.C)
+        assert oracle.near_tie(db, ds).all(), "the encoders differ off a near-tie"
+
+
 @pytest.mark.parametrize("batch", [1, 16, 128, 1024])
 def test_streaming_step(batch):
     model, frames = synth.streaming_step(batch, calls=3)
