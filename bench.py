@@ -56,6 +56,7 @@ MOSHI_DELAYS = [0, 1, 1, 1, 1, 1, 1, 1]   # acoustic delay 1 (the final model's)
 NCU_TRAFFIC_PER_UNIT = {
     "k_embed_sum": (48_951, "profiles/k_embed_sum_moshi_input.md"),        # per step
     "k_encode_tc/f32": (2_467, "profiles/k_encode_tc_offline_batch.md"),   # per fp32 frame
+    "k_encode_tc/bf16": (1_165, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
     "k_decode": (1_990, "profiles/k_decode_decode_heavy.md"),              # per frame
 }
 
@@ -399,7 +400,7 @@ def run_ours(args, rank, world, local_rank):
     lat_bytes = 2048 if work.get("dtype", "f32") == "f32" else 1024
     if do_enc:
         tf = ENC_FLOP * n / (enc_avg / 1e3) / 1e12
-        tr = NCU_TRAFFIC_PER_UNIT["k_encode_tc/f32"] if work.get("dtype", "f32") == "f32" else None
+        tr = NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + work.get("dtype", "f32"))
         kernels.append({
             "kernel": "encode call (k_encode_tc + float32 re-encode)", "bound": "tensor",
             "achieved": tf, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
