@@ -426,7 +426,10 @@ def run_ours(args, rank, world, local_rank):
     if args.self_profile and do_enc:
         _, cyc = q.encode_profile(z, out=codes, stream=stream)
         total = max(cyc["cta_total"], 1)
-        kernels[0]["self_profile_share"] = {k: round(v / total, 4) for k, v in cyc.items()}
+        counts = set(q.PROFILE_COUNTS)
+        kernels[0]["self_profile_share"] = {k: round(v / total, 4) for k, v in cyc.items()
+                                            if k not in counts}
+        kernels[0]["self_profile_counts"] = {k: cyc[k] for k in q.PROFILE_COUNTS}
     launches_per_step = (2 if do_enc else 0) + (1 if do_dec else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,

@@ -137,9 +137,10 @@ int mimi_rvq_encode_ex(mimi_rvq_t h, const void *latents, int dtype, int64_t N, 
  *   6 epilogue scanning scores                   7 epilogue merge / window / re-score
  *   8 epilogue residual update                   9 epilogue latent staging, y read-out
  *  10 epilogue barrier waits                    11 whole CTA
- *  12..14 parts of 6: TMEM loads, score arithmetic, window checks and pushes
- * (counters 5..10 and 12..14 are one epilogue thread per CTA). Codes are the same as
- * mimi_rvq_encode's.
+ * (counters 5..10 are one epilogue thread per CTA), and event counts summed over the
+ * epilogue warps (not cycles): 12 32-column chunks scanned; chunks in which some lane
+ * 13 put its displaced best into the candidate list, 14 had a runner-up near the
+ * window, 15 had three or more keys near it. Codes are the same as mimi_rvq_encode's.
  */
 int mimi_rvq_encode_profile(mimi_rvq_t h, const void *latents, int dtype, int64_t N,
                             int16_t *codes, uint64_t *cycles, struct CUstream_st *stream);

@@ -216,11 +216,12 @@ class Quantizer:
     PROFILE_SLOTS = ("producer_wait_stage", "mma_wait_operands", "mma_wait_score_buffer",
                      "mma_wait_level_operand", "mma_wait_latents", "epi_wait_score_tile",
                      "epi_scan", "epi_pick", "epi_update", "epi_stage", "epi_barrier",
-                     "cta_total", "scan_tmem", "scan_math", "scan_push")
+                     "cta_total", "n_chunks", "n_displaced", "n_runner_up", "n_more")
+    PROFILE_COUNTS = ("n_chunks", "n_displaced", "n_runner_up", "n_more")
 
     def encode_profile(self, latents, out=None, stream=None):
         """Encode and return (codes, {role: cycles summed over CTAs}) from the kernel's
-        self-profile."""
+        self-profile; the PROFILE_COUNTS entries are event counts, not cycles."""
         import torch
         n, dt = self._latents(latents)
         out = self._codes_out(n, out)

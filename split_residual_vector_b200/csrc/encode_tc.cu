@@ -73,11 +73,6 @@ constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
 // ||bf16(r)|| ||bf16(c)||, twice the need), and the float32 score
 // ||c||^2 - 2 acc rounds once more (2^-21 of its magnitude, with slack).
 // E bounds |bf16 score - exact score| for every codeword.
-// Fine-grained timing of the scan loop (profile slots 12..14). Off by default:
-// the clock reads sit in the innermost loop.
-#ifndef MIMI_SCAN_TIMING
-#define MIMI_SCAN_TIMING 0
-#endif
 
 constexpr float kAccRel = 6.103515625e-05f;         // 2^-14
 constexpr float kScoreRel = 4.76837158203125e-07f;  // 2^-21
@@ -96,7 +91,8 @@ __device__ __forceinline__ float key_lower(float k) {
 }
 
 // Optional self-profile: cycles each role spends waiting or working, summed
-// over CTAs into prof[kProfSlots] (diagnostic entry point only).
+// over CTAs into prof[kProfSlots], and counts of the scan's slower branches
+// (diagnostic entry point only; the production instantiation has none of it).
 enum ProfSlot {
     P_PROD_EMPTY = 0,   // producer waiting for a free ring stage
     P_MMA_FULL,         // MMA waiting for codebook / weight tiles
@@ -110,9 +106,10 @@ enum ProfSlot {
     P_EPI_STAGE,        // epilogue latent staging and y read-out
     P_EPI_ESYNC,        // epilogue barrier waits
     P_CTA_TOTAL,        // whole CTA
-    P_SCAN_TMEM,        // part of P_EPI_SCAN: TMEM loads of score tiles
-    P_SCAN_MATH,        // part of P_EPI_SCAN: scores, group and chunk minima
-    P_SCAN_PUSH,        // part of P_EPI_SCAN: window checks and list pushes
+    P_N_CHUNK,          // event counts, summed over epilogue warps: 32-column chunks scanned,
+    P_N_DEM,            //   chunks where some lane's displaced best entered the list,
+    P_N_SECOND,         //   chunks where some lane had a runner-up near the window,
+    P_N_MORE,           //   chunks where some lane had three or more keys near it
     kProfSlots = 16
 };
 
@@ -197,6 +194,15 @@ __device__ __forceinline__ void top2_of_32(const float (&k)[32], float& c1, floa
     c2 = H[0];
 }
 
+// Cycle counter of the self-profile; without it the counters fold away, so
+// the production kernel carries no profiling registers.
+template <bool kProf>
+__device__ __forceinline__ long long pclock() {
+    if constexpr (kProf) return clock64();
+    return 0;
+}
+
+template <bool kProf>
 __global__ void __launch_bounds__(kThreads, 1)
     k_encode_tc(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_Whi,
                 const __grid_constant__ CUtensorMap tm_Wlo, const float* __restrict__ C32,
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const long long t_cta0 = clock64();
+    const long long t_cta0 = pclock<kProf>();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -265,9 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto load = [&](const CUtensorMap* tm, int x, int y) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                const long long t0 = clock64();
+                const long long t0 = pclock<kProf>();
                 const bool r = mbar_wait(&bars->empty[s], ph ^ 1, abort, err);
-                p_empty += clock64() - t0;
+                p_empty += pclock<kProf>() - t0;
                 if (!r) return false;
                 mbar_arrive_expect_tx(&bars->full[s], STAGE_BYTES);
                 tma_load_2d(smem + RING_OFF + s * STAGE_BYTES, tm, &bars->full[s], x, y);
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t first = it > STAGES ? it - STAGES : 0;
             for (uint32_t j = first; j < it; ++j)
                 mbar_wait(&bars->full[j % STAGES], (j / STAGES) & 1, abort, err);
-            if (prof) atomicAdd(prof + P_PROD_EMPTY, (unsigned long long)p_empty);
+            if (kProf && prof) atomicAdd(prof + P_PROD_EMPTY, (unsigned long long)p_empty);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -298,9 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             long long p_full = 0, p_tempty = 0, p_afull = 0, p_zfull = 0;
             auto twait = [&](uint64_t* bar, uint32_t parity, long long& acc) {
-                const long long t0 = clock64();
+                const long long t0 = pclock<kProf>();
                 const bool r = mbar_wait(bar, parity, abort, err);
-                acc += clock64() - t0;
+                acc += pclock<kProf>() - t0;
                 return r;
             };
             for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // drain: every issued MMA must complete before TMEM is freed
             umma_commit(&bars->drain);
             mbar_wait(&bars->drain, 0, abort, err);
-            if (prof) {
+            if (kProf && prof) {
                 atomicAdd(prof + P_MMA_FULL, (unsigned long long)p_full);
                 atomicAdd(prof + P_MMA_TEMPTY, (unsigned long long)p_tempty);
                 atomicAdd(prof + P_MMA_AFULL, (unsigned long long)p_afull);
@@ -409,11 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         unsigned long long done = 0;
         long long p_tfull = 0, p_scan = 0, p_pick = 0, p_update = 0, p_stage = 0, p_esync = 0;
-        long long p_stmem = 0, p_smath = 0, p_spush = 0;
-        long long t_mark = clock64();
+        unsigned long long n_chunk = 0, n_dem = 0, n_sec = 0, n_more = 0;
+        long long t_mark = pclock<kProf>();
         // attribute the cycles since the last mark to one counter
         auto mark = [&](long long& acc) {
-            const long long t = clock64();
+            const long long t = pclock<kProf>();
             acc += t - t_mark;
             t_mark = t;
         };
@@ -448,9 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ephase = 0;
         auto esync = [&]() {
             mbar_arrive(&bars->ebar);
-            const long long t0 = clock64();
+            const long long t0 = pclock<kProf>();
             const bool r = mbar_wait(&bars->ebar, ephase & 1, abort, err);
-            p_esync += clock64() - t0;
+            p_esync += pclock<kProf>() - t0;
             ++ephase;
             return __all_sync(0xffffffffu, r) != 0;
         };
@@ -573,15 +579,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     uint32_t v[2][32];
-                    long long ts0 = MIMI_SCAN_TIMING ? clock64() : 0;
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64, v[0]);
                     tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64 + 32, v[1]);
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
-                    long long ts1 = MIMI_SCAN_TIMING ? clock64() : 0;
-                    p_stmem += ts1 - ts0;
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
                         const int k0 = nt * BN + half * 64 + c2 * 32;
@@ -596,10 +599,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             kk[4 * q4 + 3] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w), 4 * q4 + 3);
                         }
                         const float c1k = min_of_32(kk);
-                        if (MIMI_SCAN_TIMING) {
-                            ts0 = clock64();
-                            p_smath += ts0 - ts1;
-                        }
                         const float g1 = globalize(c1k, k0);
                         // the key that loses the best slot (or the chunk minimum, if it
                         // does not take it) joins the list when it is inside the window
@@ -608,13 +607,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float thr = cs.best + key_slack(cs.best) + twoE;
                         const float inf = __int_as_float(0x7f800000);
                         const bool dem_in = key_lower(dem) <= thr;
-                        if (__any_sync(0xffffffffu, dem_in)) cands_insert(cs, dem_in ? dem : inf);
+                        if (kProf) ++n_chunk;
+                        if (__any_sync(0xffffffffu, dem_in)) {
+                            if (kProf) ++n_dem;
+                            cands_insert(cs, dem_in ? dem : inf);
+                        }
                         // Any other key of the chunk inside the window? On the FMA pipe:
                         // sum_j sat(kd (Td - key_j)), minus the minimum's own term. Td widens
                         // thr by more than the key perturbations, and every key below Td adds
                         // at least 2^-16, far above the rounding of the sum (<= 2^-18).
                         const float Td = thr + 1.953125e-3f * (fabsf(thr) + twoE);
-                        const float kd = 16.f / (fabsf(Td) + twoE + 1e-30f);
+                        const float kd = __fdividef(16.f, fabsf(Td) + twoE + 1e-30f);
                         const float K = fmaf(kd, Td, 1.52587890625e-05f);
                         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
@@ -627,6 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float other = ((a0 + a1) + (a2 + a3)) - fma_sat(-kd, c1k, K);
                         const bool second_cand = other > 9.5367431640625e-07f;  // 2^-20
                         if (__any_sync(0xffffffffu, second_cand)) {
+                            if (kProf) ++n_sec;
                             // some lane has another key near the window: its runner-up goes
                             // in, and a third key is looked for only if the sum says so
                             float c1b, c2k;
@@ -637,17 +641,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const bool more = second_cand &&
                                               (other - fma_sat(-kd, c2k, K)) > 9.5367431640625e-07f;
                             if (__any_sync(0xffffffffu, more)) {
+                                if (kProf) ++n_more;
+                                // further keys in ascending order (the keys are distinct: they
+                                // carry their position), while they are inside the window
+                                float last = c2k;
+                                bool go = more;
+#pragma unroll 1
+                                for (int t = 0; t < TOPK - 2 && __any_sync(0xffffffffu, go); ++t) {
+                                    float nk[32];
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) {
-                                    const float gj = globalize(kk[j], k0);
-                                    const bool in = more && gj != g1 && gj != g2 && key_lower(gj) <= thr;
-                                    cands_insert(cs, in ? gj : inf);
+                                    for (int j = 0; j < 32; ++j) nk[j] = kk[j] > last ? kk[j] : inf;
+                                    const float mn = min_of_32(nk);
+                                    const float gn = globalize(mn, k0);
+                                    const bool in = go && mn < inf && key_lower(gn) <= thr;
+                                    cands_insert(cs, in ? gn : inf);
+                                    go = in;
+                                    last = mn;
                                 }
+                                // a chunk with more window keys than the list holds: what was
+                                // not taken counts as evicted, so the row is not certified
+                                if (go) cs.evicted = fminf(cs.evicted, globalize(last, k0));
                             }
-                        }
-                        if (MIMI_SCAN_TIMING) {
-                            ts1 = clock64();
-                            p_spush += ts1 - ts0;
                         }
                     }
                 }
@@ -807,16 +821,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         mark(p_stage);
-        if (prof && warp == 2 && lane == 0) {
+        if (kProf && prof && warp == 2 && lane == 0) {
             atomicAdd(prof + P_EPI_TFULL, (unsigned long long)p_tfull);
             atomicAdd(prof + P_EPI_SCAN, (unsigned long long)p_scan);
             atomicAdd(prof + P_EPI_PICK, (unsigned long long)p_pick);
             atomicAdd(prof + P_EPI_UPDATE, (unsigned long long)p_update);
             atomicAdd(prof + P_EPI_STAGE, (unsigned long long)p_stage);
             atomicAdd(prof + P_EPI_ESYNC, (unsigned long long)p_esync);
-            atomicAdd(prof + P_SCAN_TMEM, (unsigned long long)p_stmem);
-            atomicAdd(prof + P_SCAN_MATH, (unsigned long long)p_smath);
-            atomicAdd(prof + P_SCAN_PUSH, (unsigned long long)p_spush);
+        }
+        if (kProf && prof && lane == 0) {
+            atomicAdd(prof + P_N_CHUNK, n_chunk);
+            atomicAdd(prof + P_N_DEM, n_dem);
+            atomicAdd(prof + P_N_SECOND, n_sec);
+            atomicAdd(prof + P_N_MORE, n_more);
         }
         // count frames (one atomic per warp)
         for (int o = 16; o > 0; o >>= 1) done += __shfl_xor_sync(0xffffffffu, done, o);
@@ -826,14 +843,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
-    if (prof && threadIdx.x == 0)
-        atomicAdd(prof + P_CTA_TOTAL, (unsigned long long)(clock64() - t_cta0));
+    if (kProf && prof && threadIdx.x == 0)
+        atomicAdd(prof + P_CTA_TOTAL, (unsigned long long)(pclock<kProf>() - t_cta0));
 }
 
 }  // namespace
 
 cudaError_t encode_tc_configure() {
-    return cudaFuncSetAttribute(k_encode_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(
+        k_encode_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_encode_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SMEM_BYTES);
 }
 
@@ -843,10 +863,10 @@ cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t 
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + BM - 1) / BM;
     const int grid = (int)(tiles < max_ctas ? tiles : max_ctas);
-    k_encode_tc<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm,
-                                                   t.cbound, z, dtype, n, n_q, variant, codes,
-                                                   y_out, t.err, t.rescan_count, t.rescan_list,
-                                                   t.stats, prof);
+    auto* kernel = prof ? k_encode_tc<true> : k_encode_tc<false>;
+    kernel<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm, t.cbound,
+                                              z, dtype, n, n_q, variant, codes, y_out, t.err,
+                                              t.rescan_count, t.rescan_list, t.stats, prof);
     return cudaGetLastError();
 }
 

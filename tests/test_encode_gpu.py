@@ -257,6 +257,47 @@ def test_many_equal_codewords_go_to_the_full_scan():
     assert rescanned == 3
 
 
+@pytest.mark.parametrize("k", [3, 5, 7, 8, 11])
+def test_equal_codewords_inside_one_scan_chunk(k):
+    """k identical codewords in one 32-codeword chunk of the semantic codebook (columns 64..95),
+    nearest to the frame: the scan takes them from the chunk in ascending key order. Up to 7
+    fit the candidate list and certify without a re-encode; with more than the list holds the
+    row is re-encoded by the float32 full scan. Either way the lowest tied index wins."""
+    model = _small_model(35)
+    tied = [64 + 3 * j for j in range(k)]
+    for j in tied:
+        model.C[0, j] = model.C[0, tied[0]]
+    q = quantizer(model)
+    z = np.stack([synth.plant_latent(model, {0: tied[-1]})] * 3)
+    codes = q.encode(to_device(z)).cpu().numpy()
+    assert q.get_error() == 0
+    assert (codes[:, 0] == tied[0]).all()
+    ref, _, _ = oracle.encode(z, model.W_in, model.C)
+    assert (ref[:, 0] == tied[0]).all()
+    _, rescanned = q.stats()
+    if k <= 7:
+        assert rescanned == 0
+    elif k > 8:
+        assert rescanned == 3
+
+
+def test_self_profile_counts(offline_small):
+    """The diagnostic entry point returns the same codes, cycle counters for every role, and
+    branch counts that respect their nesting; one count per 32-column chunk scanned by each
+    epilogue warp (8 warps x 2 chunks x 16 tiles x 8 codebooks per 128-frame tile)."""
+    work, q = offline_small
+    z = to_device(work.z)
+    codes = q.encode(z).cpu().numpy()
+    pcodes, prof = q.encode_profile(z)
+    assert q.get_error() == 0
+    assert np.array_equal(pcodes.cpu().numpy(), codes)
+    tiles = (len(work.z) + 127) // 128
+    assert prof["n_chunks"] == tiles * 8 * 2 * 16 * 8
+    assert prof["n_chunks"] >= prof["n_displaced"] >= 0
+    assert prof["n_chunks"] >= prof["n_runner_up"] >= prof["n_more"] >= 0
+    assert prof["cta_total"] > 0 and prof["epi_scan"] > 0
+
+
 def test_rescan_of_many_frames_in_several_batches():
     """Every level-1 codeword has ~20 exact copies, so no frame's candidate window can be
     certified and all 2500 frames are re-encoded by the float32 wide encoder, 1024 at a time
