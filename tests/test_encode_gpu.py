@@ -242,11 +242,11 @@ def test_duplicated_codewords_pick_the_lowest_index():
 
 
 def test_many_equal_codewords_go_to_the_full_scan():
-    """Twelve identical codewords nearest to the frame: more ties than the top-8 can hold, so
-    the candidate set cannot be certified; the frame must be re-encoded by the full scan and
-    still return the lowest of the tied indices."""
+    """Twenty identical codewords nearest to the frame, spread over the codebook: more ties
+    than the candidate list holds, so the candidate set cannot be certified; the frame must be
+    re-encoded by the full scan and still return the lowest of the tied indices."""
     model = _small_model(33)
-    tied = [100 + 37 * j for j in range(12)]
+    tied = [100 + 37 * j for j in range(20)]
     for j in tied:
         model.C[0, j] = model.C[0, tied[0]]
     q = quantizer(model)
@@ -257,14 +257,15 @@ def test_many_equal_codewords_go_to_the_full_scan():
     assert rescanned == 3
 
 
-@pytest.mark.parametrize("k", [3, 5, 7, 8, 11])
+@pytest.mark.parametrize("k", [3, 5, 7, 8, 11, 20])
 def test_equal_codewords_inside_one_scan_chunk(k):
     """k identical codewords in one 32-codeword chunk of the semantic codebook (columns 64..95),
     nearest to the frame: the scan takes them from the chunk in ascending key order. Up to 7
-    fit the candidate list and certify without a re-encode; with more than the list holds the
-    row is re-encoded by the float32 full scan. Either way the lowest tied index wins."""
+    fit the candidate list and certify without a re-encode; twenty are more than the list
+    holds, and the row is re-encoded by the float32 full scan. Either way the lowest tied
+    index wins."""
     model = _small_model(35)
-    tied = [64 + 3 * j for j in range(k)]
+    tied = [64 + (3 * j if k <= 11 else j) for j in range(k)]
     for j in tied:
         model.C[0, j] = model.C[0, tied[0]]
     q = quantizer(model)
@@ -277,7 +278,7 @@ def test_equal_codewords_inside_one_scan_chunk(k):
     _, rescanned = q.stats()
     if k <= 7:
         assert rescanned == 0
-    elif k > 8:
+    elif k == 20:
         assert rescanned == 3
 
 
