@@ -4,7 +4,9 @@ A step is one pass of the whole hot path over one batch: encode (projection,
 semantic VQ, 7-level acoustic RVQ, codes) and decode (gather-sum, projection back)
 of the offline-batch workload: 64 streams x 3750 frames = 240 000 fp32 frames.
 Other workloads (--workload) are the 1 048 576-frame bf16 bulk encode, the
-1 048 576-frame decode-heavy decode, and the streaming step.
+1 048 576-frame decode-heavy decode, the streaming step and the Moshi input
+(delay packing + embedding sum). --n-q uses only the first n_q codebooks and
+--variant 1 runs the acoustic RVQ on y - S_s (encode and decode workloads).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 torch.cuda.synchronize(), timed with CUDA events on the stream the kernels run
@@ -12,6 +14,7 @@ on; the max over ranks is reported. Inputs are larger than L2 (they are not
 re-read from L2 between steps). One JSON line is printed by rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--n-q Q] [--variant V]
 """
 from __future__ import annotations
 
@@ -33,9 +36,18 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 FRAME_HZ = 12.5
-ENC_FLOP = 8 * 2 * 2048 * 256 + 2 * 256 * 512     # 8 650 752 per frame
-DEC_FLOP = 2 * 512 * 256                         # 262 144 per frame (+ 1 792 adds)
-DEC_BYTES = 8 * 2 + 512 * 4                      # codes in + fp32 latents out
+
+
+def enc_flop(n_q=8):
+    """Scores of n_q codebooks plus the 512 -> 256 projection, per frame (8 650 752 at 8)."""
+    return n_q * 2 * 2048 * 256 + 2 * 256 * 512
+
+
+def dec_bytes(n_q=8):
+    """n_q int16 codes in, 512 fp32 out, per frame (2 064 at 8)."""
+    return n_q * 2 + 512 * 4
+
+
 METRIC = "RVQ encode/decode frames/s (real-time streams @12.5 Hz) and % of roofline, 1xB200"
 
 WORKLOADS = {
@@ -246,9 +258,9 @@ def to_device_latents(torch, z, dtype, device):
     return torch.from_numpy(z).to(device)
 
 
-def cpu_baseline(work, name, budget_s=12.0):
+def cpu_baseline(work, name, budget_s=12.0, n_q=8, variant=0):
     """The float64 oracle on this host's cores over a bounded sample of the workload, and the
-    same on one thread over a small slice."""
+    same on one thread over a small slice (with the run's n_q and variant)."""
     import oracle
     m = work["model"]
     cores = oracle.threads(0)
@@ -256,11 +268,13 @@ def cpu_baseline(work, name, budget_s=12.0):
     def run(n, nthreads=0):
         t0 = time.perf_counter()
         if name in ("offline_batch", "bulk_tokenization"):
-            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C, nthreads=nthreads)
+            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C, n_q=n_q, variant=variant,
+                                        nthreads=nthreads)
             if name == "offline_batch":
                 oracle.decode(codes, m.C, m.W_out, nthreads=nthreads)
         else:
-            oracle.decode(work["codes"][:n], m.C, m.W_out, nthreads=nthreads)
+            oracle.decode(np.ascontiguousarray(work["codes"][:n, :n_q]), m.C, m.W_out,
+                          nthreads=nthreads)
         return time.perf_counter() - t0
 
     n = 64 if name != "decode_heavy" else 4096
@@ -296,11 +310,12 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
     do_enc = name in ("offline_batch", "bulk_tokenization")
     do_dec = name in ("offline_batch", "decode_heavy")
+    n_q, variant = args.n_q, args.variant
     if do_enc:
         z = to_device_latents(torch, work["z"], work["dtype"], device)
-        codes = torch.empty((n, 8), dtype=torch.int16, device=device)
+        codes = torch.empty((n, n_q), dtype=torch.int16, device=device)
     else:
-        codes = torch.from_numpy(work["codes"]).to(device)
+        codes = torch.from_numpy(np.ascontiguousarray(work["codes"][:, :n_q])).to(device)
     x = torch.empty((n, 512), dtype=torch.float32, device=device) if do_dec else None
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -310,7 +325,7 @@ def run_ours(args, rank, world, local_rank):
         if do_enc:
             a, b = ev(), ev()
             a.record(stream)
-            q.encode(z, out=codes, stream=stream)
+            q.encode(z, n_q=n_q, variant=variant, out=codes, stream=stream)
             b.record(stream)
             if timed:
                 enc_ms.append((a, b))
@@ -351,7 +366,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_e2e:
         k = max(4, min(args.steps, 10))
         # two sets of device buffers; the host side holds one input and two result buffers
-        h_codes = [torch.empty((n, 8), dtype=torch.int16, pin_memory=True) for _ in range(2)]
+        h_codes = [torch.empty((n, n_q), dtype=torch.int16, pin_memory=True) for _ in range(2)]
         h_x = ([torch.empty((n, 512), dtype=torch.float32, pin_memory=True) for _ in range(2)]
                if do_dec else None)
         codes2 = [codes, torch.empty_like(codes)]
@@ -372,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
 
         def compute(b, s):
             if do_enc:
-                q.encode(in2[b], out=codes2[b], stream=s)
+                q.encode(in2[b], n_q=n_q, variant=variant, out=codes2[b], stream=s)
             if do_dec:
                 q.decode(codes2[b], out=x2[b], stream=s)
 
@@ -399,31 +414,34 @@ def run_ours(args, rank, world, local_rank):
     kernels = []
     lat_bytes = 2048 if work.get("dtype", "f32") == "f32" else 1024
     if do_enc:
-        tf = ENC_FLOP * n / (enc_avg / 1e3) / 1e12
-        tr = NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + work.get("dtype", "f32"))
+        tf = enc_flop(n_q) * n / (enc_avg / 1e3) / 1e12
+        # the captured DRAM traffic is for the full 8-codebook, variant-0 encode
+        tr = (NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + work.get("dtype", "f32"))
+              if (n_q, variant) == (8, 0) else None)
         kernels.append({
             "kernel": "encode call (k_encode_tc + float32 re-encode)", "bound": "tensor",
             "achieved": tf, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
             "frac": tf / peaks["bf16_tflops_sustained"],
             "traffic": tr[0] * n if tr else None, "traffic_source": tr[1] if tr else None,
             "ms": enc_avg,
-            "algorithmic": f"{ENC_FLOP} FLOP/frame x {n} frames; HBM {lat_bytes + 16} B/frame",
-            "hbm_gbs": (lat_bytes + 16) * n / (enc_avg / 1e3) / 1e9})
+            "algorithmic": (f"{enc_flop(n_q)} FLOP/frame x {n} frames; "
+                            f"HBM {lat_bytes + 2 * n_q} B/frame"),
+            "hbm_gbs": (lat_bytes + 2 * n_q) * n / (enc_avg / 1e3) / 1e9})
     if do_dec:
-        gbs = DEC_BYTES * n / (dec_avg / 1e3) / 1e9
-        tr = NCU_TRAFFIC_PER_UNIT["k_decode"]
+        gbs = dec_bytes(n_q) * n / (dec_avg / 1e3) / 1e9
+        tr = NCU_TRAFFIC_PER_UNIT["k_decode"] if n_q == 8 else None
         kernels.append({
             "kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": tr[0] * n,
-            "traffic_source": tr[1], "ms": dec_avg,
-            "algorithmic": f"{DEC_BYTES} B/frame x {n} frames (codes in, fp32 latents out)"})
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": tr[0] * n if tr else None,
+            "traffic_source": tr[1] if tr else None, "ms": dec_avg,
+            "algorithmic": f"{dec_bytes(n_q)} B/frame x {n} frames (codes in, fp32 latents out)"})
     dominant = kernels[0]
     roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = dominant["kernel"]
     roofline["traffic_source"] = dominant.get("traffic_source")
     roofline["peak_source"] = (f"{peaks['source']} "
                                f"{'bf16_tflops_sustained' if dominant['bound'] == 'tensor' else 'hbm_gbs'}")
-    if args.self_profile and do_enc:
+    if args.self_profile and do_enc and (n_q, variant) == (8, 0):
         _, cyc = q.encode_profile(z, out=codes, stream=stream)
         total = max(cyc["cta_total"], 1)
         counts = set(q.PROFILE_COUNTS)
@@ -438,7 +456,8 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16 products, f32 accumulate/re-score", "data": "synthetic",
         "config": {"workload": f"{name}: {WORKLOADS[name]}" + (
                        f" (reduced to {n} frames)" if args.frames else ""), "frames_per_gpu": n,
-                   "latent_dtype": work.get("dtype"), "parallelism": f"replicas x{world}",
+                   "latent_dtype": work.get("dtype"), "n_q": n_q, "variant": variant,
+                   "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (not re-read from L2 between steps)"},
         "realtime_streams": value / FRAME_HZ,
         "roofline": roofline, "kernels": kernels,
@@ -446,7 +465,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(), "status": status, "e2e": e2e,
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(work, name)
+        line["cpu_baseline"] = cpu_baseline(work, name, n_q=n_q, variant=variant)
     if dist:
         dist.destroy_process_group()
     return line
@@ -667,11 +686,12 @@ def run_reference(args):
             return
         m = work["model"]
         if name in ("offline_batch", "bulk_tokenization", "streaming"):
-            c, _, _ = oracle.encode(work["z"][:nf], m.W_in, m.C)
+            c, _, _ = oracle.encode(work["z"][:nf], m.W_in, m.C, n_q=args.n_q,
+                                    variant=args.variant)
             if name == "offline_batch":
                 oracle.decode(c, m.C, m.W_out)
         else:
-            oracle.decode(work["codes"][:nf], m.C, m.W_out)
+            oracle.decode(np.ascontiguousarray(work["codes"][:nf, :args.n_q]), m.C, m.W_out)
 
     t0 = time.perf_counter()
     one(32)
@@ -691,7 +711,10 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{name}: {WORKLOADS[name]}", "sample_frames": nf},
+            "config": {"workload": f"{name}: {WORKLOADS[name]}", "sample_frames": nf,
+                       **({"n_q": args.n_q, "variant": args.variant}
+                          if name in ("offline_batch", "bulk_tokenization", "decode_heavy")
+                          else {})},
             "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0,
@@ -712,6 +735,11 @@ def main():
                     help="add the encode kernel's per-role cycle shares (one extra untimed call)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n-q", type=int, default=8, choices=range(1, 9),
+                    help="codebooks used (encode/decode workloads): the semantic one and "
+                         "n_q - 1 acoustic levels")
+    ap.add_argument("--variant", type=int, default=0, choices=(0, 1),
+                    help="encode workloads: 1 runs the acoustic RVQ on y - S_s")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
