@@ -60,3 +60,25 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_roofline_work_per_frame():
+    """The roofline's algorithmic work per frame, at every n_q: scores of n_q codebooks of
+    2048 x 256 plus the 512 -> 256 projection; n_q int16 codes in and 512 fp32 out for decode."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.enc_flop() == 8 * 2 * 2048 * 256 + 2 * 256 * 512 == 8_650_752
+    assert bench.dec_bytes() == 2_064
+    for n_q in range(1, 9):
+        assert bench.enc_flop(n_q) - bench.enc_flop(n_q - 1) == 2 * 2048 * 256
+        assert bench.dec_bytes(n_q) == 2 * n_q + 2048
+
+
+def test_bench_options():
+    """--n-q and --variant reach the encode calls; out-of-range values are refused."""
+    run = lambda *a: subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *a],  # noqa: E731
+                                    capture_output=True, text=True, timeout=120)
+    out = run("--help")
+    assert out.returncode == 0 and "--n-q" in out.stdout and "--variant" in out.stdout
+    assert run("--n-q", "9").returncode != 0
+    assert run("--variant", "2").returncode != 0
