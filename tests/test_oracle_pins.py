@@ -9,7 +9,12 @@ Which plausible mistake each pin catches:
     direction (a transposed W_in cannot map pinv(W_in) y back to y);
   * identity projection: projection indexing (rows vs columns of W_in);
   * decode invariants: a dropped codebook in the sum, a transposed W_out;
-  * rates: the golden tables the pages print.
+  * rates: the golden tables the pages print;
+  * translation invariance of the distance: a score without the ||c||^2 term, a chain fed
+    from the wrong vector (checked by planting -2 r.c as the score in the oracle: both
+    variants fail);
+  * codeword relabelling: an index or row-offset mistake (checked by planting a row offset
+    of one: the pin fails).
 """
 import itertools
 import os
@@ -338,3 +343,51 @@ def test_near_tie_rule():
     assert oracle.near_tie(db, ds).tolist() == [False, False]
     ds[0, 0] = 10.0 + 1e-4
     assert oracle.near_tie(db, ds).tolist() == [True, False]
+
+
+# ----------------------------------------------------------- invariances of the distance
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+def test_translation_invariance(variant):
+    """Squared distances do not change when the target and every candidate move by the same
+    vector t. Variant 0 quantises y with codebook 0 and with the acoustic chain from codebook 1,
+    so shifting y, codebook 0 and codebook 1 by t leaves every code and distance as it was;
+    variant 1 feeds the chain y - S_s, so shifting y and codebook 0 alone does. Integer data
+    keep every float64 operation exact, ties included. Catches a score without the ||c||^2 term
+    (-2 y.c alone is not translation invariant) and a chain fed from the wrong vector."""
+    rng = np.random.default_rng(41 + variant)
+    Q, K, D, N = 4, 24, 6, 40
+    C = rng.integers(-6, 7, size=(Q, K, D)).astype(np.float32)
+    y = rng.integers(-9, 10, size=(N, D)).astype(np.float64)
+    t = rng.integers(-20, 21, size=D)
+    C2 = C.copy()
+    C2[0] += t
+    if variant == 0:
+        C2[1] += t
+    codes, db, ds = oracle.encode_projected(y, C, variant=variant)
+    codes2, db2, ds2 = oracle.encode_projected(y + t, C2, variant=variant)
+    assert np.array_equal(codes, codes2)
+    assert np.array_equal(db, db2) and np.array_equal(ds, ds2)
+    # and the plain shift of y alone does move the codes (the data are not degenerate)
+    codes3, _, _ = oracle.encode_projected(y + t, C, variant=variant)
+    assert not np.array_equal(codes, codes3)
+
+
+def test_codeword_permutation_equivariance():
+    """Relabelling the codewords of every codebook relabels the codes the same way and leaves
+    the distances bit for bit unchanged. Catches an index or row-offset mistake in the scan."""
+    rng = np.random.default_rng(43)
+    Q, K, D, N = 8, 64, 16, 200
+    C = rng.standard_normal((Q, K, D)).astype(np.float32)
+    for level in range(1, Q):
+        C[level] *= 0.5 ** level
+    y = rng.standard_normal((N, D))
+    perms = [rng.permutation(K) for _ in range(Q)]       # new index j holds old codeword p[j]
+    Cp = np.stack([C[level][perms[level]] for level in range(Q)])
+    codes, db, ds = oracle.encode_projected(y, C)
+    codes_p, db_p, ds_p = oracle.encode_projected(y, Cp)
+    inverse = [np.argsort(p) for p in perms]
+    for level in range(Q):
+        assert np.array_equal(codes_p[:, level], inverse[level][codes[:, level]])
+    assert np.array_equal(db, db_p) and np.array_equal(ds, ds_p)
