@@ -1,17 +1,25 @@
 """Benchmark of the B200 split-RVQ hot path (Mimi tokenizer bottleneck).
 
-A step is one pass of the whole hot path over one batch: encode (projection,
-semantic VQ, 7-level acoustic RVQ, codes) and decode (gather-sum, projection back)
-of the offline-batch workload: 64 streams x 3750 frames = 240 000 fp32 frames.
-Other workloads (--workload) are the 1 048 576-frame bf16 bulk encode, the
-1 048 576-frame decode-heavy decode, the streaming step and the Moshi input
-(delay packing + embedding sum). --n-q uses only the first n_q codebooks and
---variant 1 runs the acoustic RVQ on y - S_s (encode and decode workloads).
+A step is one pass of the whole hot path: the encode of 1 048 576 bf16 frames (bulk
+tokenization: projection, semantic VQ, 7-level acoustic RVQ, codes) and the decode of
+1 048 576 frames of codes (decode-heavy: gather-sum of the chosen codewords and the
+projection back), each on its own seeded model. Other workloads (--workload) are the
+240 000-frame fp32 offline batch (encode, then decode of its codes), either 1M-frame half
+alone, the streaming step and the Moshi input (delay packing + embedding sum). --n-q uses
+only the first n_q codebooks and --variant 1 runs the acoustic RVQ on y - S_s (encode and
+decode workloads).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 torch.cuda.synchronize(), timed with CUDA events on the stream the kernels run
 on; the max over ranks is reported. Inputs are larger than L2 (they are not
-re-read from L2 between steps). One JSON line is printed by rank 0.
+re-read from L2 between steps). One JSON line is printed by rank 0. Each call is
+timed alone with its own events, so its roofline fraction is taken against the
+burst peak (a kernel timed in isolation); the sustained peak applies only to a
+region that runs for seconds.
+
+--gpus N runs N replicas (one process per GPU, weak scaling). Under torchrun the
+world size must equal N; without torchrun and N > 1 the script launches itself
+under torch.distributed.run with N processes.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
                     [--n-q Q] [--variant V]
@@ -51,6 +59,10 @@ def dec_bytes(n_q=8):
 METRIC = "RVQ encode/decode frames/s (real-time streams @12.5 Hz) and % of roofline, 1xB200"
 
 WORKLOADS = {
+    "encode_decode_1m": "encode of 1048576 bf16 frames [1048576,512] to int16 codes "
+                        "[1048576,8] (bulk tokenization) + decode of 1048576 frames of codes "
+                        "(semantic uniform, acoustic Zipf(1.1)) to fp32 [1048576,512] "
+                        "(decode-heavy); each half on its own seeded model",
     "offline_batch": "64 streams x 3750 frames = 240000 fp32 frames; encode to int16 codes "
                      "[240000,8] then decode to fp32 [240000,512]",
     "bulk_tokenization": "1048576 bf16 frames [1048576,512]; encode only, int16 codes out",
@@ -71,6 +83,11 @@ NCU_TRAFFIC_PER_UNIT = {
     "k_encode_tc/bf16": (1_161, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
     "k_decode": (1_990, "profiles/k_decode_decode_heavy.md"),              # per frame
 }
+
+
+# Kernel launches of this library per encode call (k_encode_tc, then the float32 re-encode
+# of the frames it could not certify) and per decode call (k_decode).
+ENCODE_LAUNCHES = 2
 
 
 def load_peaks():
@@ -237,19 +254,27 @@ def pipelined_e2e(torch, device, k, h2d, compute, d2h):
 
 def make_workload(name, rank, frames=None):
     """Host-side inputs for one rank (weak scaling: every rank gets a full workload).
-    ``frames`` shrinks the workload (profiling captures only; the bench line uses the
-    full size)."""
+
+    Returns {"enc": {model, z, dtype} or None, "dec": {model, codes} or None, "frames": n,
+    "decode_own_codes": bool}. The offline batch decodes the codes its own encode produced
+    (one model); the 1M-frame target pairs the bulk encode and the decode-heavy decode, each
+    with its own seeded model. ``frames`` shrinks the workload (profiling captures only; the
+    bench line uses the full size)."""
+    kw = {"n": frames} if frames else {}
+    enc = dec = None
     if name == "offline_batch":
-        w = synth.offline_batch(**({"n": frames} if frames else {}), seed=1 + 100 * rank)
-        return {"model": w.model, "z": w.z, "dtype": "f32", "frames": len(w.z)}
-    if name == "bulk_tokenization":
-        w = synth.bulk_tokenization(**({"n": frames} if frames else {}), seed=3 + 100 * rank)
-        return {"model": w.model, "z": w.z, "dtype": "bf16", "frames": len(w.z)}
-    if name == "decode_heavy":
-        model, codes = synth.decode_heavy(**({"n": frames} if frames else {}),
-                                          seed=4 + 100 * rank)
-        return {"model": model, "codes": codes, "frames": len(codes)}
-    raise ValueError(name)
+        w = synth.offline_batch(**kw, seed=1 + 100 * rank)
+        enc = {"model": w.model, "z": w.z, "dtype": "f32"}
+    if name in ("bulk_tokenization", "encode_decode_1m"):
+        w = synth.bulk_tokenization(**kw, seed=3 + 100 * rank)
+        enc = {"model": w.model, "z": w.z, "dtype": "bf16"}
+    if name in ("decode_heavy", "encode_decode_1m"):
+        model, codes = synth.decode_heavy(**kw, seed=4 + 100 * rank)
+        dec = {"model": model, "codes": codes}
+    if enc is None and dec is None:
+        raise ValueError(name)
+    n = len(enc["z"]) if enc is not None else len(dec["codes"])
+    return {"enc": enc, "dec": dec, "frames": n, "decode_own_codes": name == "offline_batch"}
 
 
 def to_device_latents(torch, z, dtype, device):
@@ -258,36 +283,61 @@ def to_device_latents(torch, z, dtype, device):
     return torch.from_numpy(z).to(device)
 
 
-def cpu_baseline(work, name, budget_s=12.0, n_q=8, variant=0):
-    """The float64 oracle on this host's cores over a bounded sample of the workload, and the
-    same on one thread over a small slice (with the run's n_q and variant)."""
+def oracle_step(work, nf, n_q=8, variant=0, nthreads=0):
+    """The oracle's pass over the first nf frames of each half of the workload; returns the
+    seconds spent on the encode half and on the decode half."""
     import oracle
-    m = work["model"]
-    cores = oracle.threads(0)
-
-    def run(n, nthreads=0):
+    t_enc = t_dec = 0.0
+    enc, dec = work["enc"], work["dec"]
+    codes = None
+    if enc is not None:
+        m = enc["model"]
         t0 = time.perf_counter()
-        if name in ("offline_batch", "bulk_tokenization"):
-            codes, _, _ = oracle.encode(work["z"][:n], m.W_in, m.C, n_q=n_q, variant=variant,
-                                        nthreads=nthreads)
-            if name == "offline_batch":
-                oracle.decode(codes, m.C, m.W_out, nthreads=nthreads)
-        else:
-            oracle.decode(np.ascontiguousarray(work["codes"][:n, :n_q]), m.C, m.W_out,
-                          nthreads=nthreads)
-        return time.perf_counter() - t0
+        codes, _, _ = oracle.encode(enc["z"][:nf], m.W_in, m.C, n_q=n_q, variant=variant,
+                                    nthreads=nthreads)
+        t_enc = time.perf_counter() - t0
+    if work["decode_own_codes"]:
+        m = enc["model"]
+        t0 = time.perf_counter()
+        oracle.decode(codes, m.C, m.W_out, nthreads=nthreads)
+        t_dec = time.perf_counter() - t0
+    elif dec is not None:
+        m = dec["model"]
+        t0 = time.perf_counter()
+        oracle.decode(np.ascontiguousarray(dec["codes"][:nf, :n_q]), m.C, m.W_out,
+                      nthreads=nthreads)
+        t_dec = time.perf_counter() - t0
+    return t_enc, t_dec
 
-    n = 64 if name != "decode_heavy" else 4096
-    dt = run(n)
-    n = int(max(n, min(work["frames"], n * budget_s / max(dt, 1e-3))))
-    dt = run(n)
-    n1 = 32 if name != "decode_heavy" else 4096
-    dt1 = run(n1, nthreads=1)
-    what = {"offline_batch": "encode+decode", "bulk_tokenization": "encode",
-            "decode_heavy": "decode"}[name]
-    return {"value": n / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n} frames of the workload, {what}, float64 oracle, {dt:.1f} s",
-            "one_thread": {"value": n1 / dt1, "unit": "frames/s", "sample": f"first {n1} frames"}}
+
+def _halves(work):
+    parts = []
+    if work["enc"] is not None:
+        parts.append("encode")
+    if work["decode_own_codes"] or work["dec"] is not None:
+        parts.append("decode")
+    return "+".join(parts)
+
+
+def cpu_baseline(work, budget_s=12.0, n_q=8, variant=0):
+    """The float64 oracle on this host's cores over a bounded sample of the workload, and the
+    same on one thread over a small slice (with the run's n_q and variant). A frame counts
+    once it has been through every half of the step, so the rate is 1 / (encode seconds per
+    frame + decode seconds per frame)."""
+    import oracle
+    cores = oracle.threads(0)
+    enc_only_cost = work["enc"] is not None
+    n = 64 if enc_only_cost else 4096
+    te, td = oracle_step(work, n, n_q, variant)
+    n = int(max(n, min(work["frames"], n * budget_s / max(te + td, 1e-3))))
+    te, td = oracle_step(work, n, n_q, variant)
+    n1 = 32 if enc_only_cost else 4096
+    te1, td1 = oracle_step(work, n1, n_q, variant, nthreads=1)
+    return {"value": n / (te + td), "unit": "frames/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} frames of each half ({_halves(work)}), float64 oracle, "
+                      f"{te:.1f} s encode + {td:.1f} s decode",
+            "one_thread": {"value": n1 / (te1 + td1), "unit": "frames/s",
+                           "sample": f"first {n1} frames"}}
 
 
 # --------------------------------------------------------------------- our arm
@@ -303,20 +353,27 @@ def run_ours(args, rank, world, local_rank):
 
     name = args.workload
     work = make_workload(name, rank, args.frames)
-    m = work["model"]
-    q = pkg.Quantizer(torch.from_numpy(m.C).to(device), torch.from_numpy(m.W_in).to(device),
-                      torch.from_numpy(m.W_out).to(device))
+    enc, dec = work["enc"], work["dec"]
     n = work["frames"]
-    stream = torch.cuda.current_stream(device)
-    do_enc = name in ("offline_batch", "bulk_tokenization")
-    do_dec = name in ("offline_batch", "decode_heavy")
     n_q, variant = args.n_q, args.variant
+    do_enc = enc is not None
+    do_dec = work["decode_own_codes"] or dec is not None
+
+    def handle(m):
+        return pkg.Quantizer(torch.from_numpy(m.C).to(device), torch.from_numpy(m.W_in).to(device),
+                             torch.from_numpy(m.W_out).to(device))
+
+    q_enc = handle(enc["model"]) if do_enc else None
+    q_dec = q_enc if work["decode_own_codes"] else (handle(dec["model"]) if do_dec else None)
+    stream = torch.cuda.current_stream(device)
+    z = codes = dcodes = x = None
     if do_enc:
-        z = to_device_latents(torch, work["z"], work["dtype"], device)
+        z = to_device_latents(torch, enc["z"], enc["dtype"], device)
         codes = torch.empty((n, n_q), dtype=torch.int16, device=device)
-    else:
-        codes = torch.from_numpy(np.ascontiguousarray(work["codes"][:, :n_q])).to(device)
-    x = torch.empty((n, 512), dtype=torch.float32, device=device) if do_dec else None
+    if do_dec:
+        dcodes = (codes if work["decode_own_codes"] else
+                  torch.from_numpy(np.ascontiguousarray(dec["codes"][:, :n_q])).to(device))
+        x = torch.empty((n, 512), dtype=torch.float32, device=device)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     enc_ms, dec_ms = [], []
@@ -325,14 +382,14 @@ def run_ours(args, rank, world, local_rank):
         if do_enc:
             a, b = ev(), ev()
             a.record(stream)
-            q.encode(z, n_q=n_q, variant=variant, out=codes, stream=stream)
+            q_enc.encode(z, n_q=n_q, variant=variant, out=codes, stream=stream)
             b.record(stream)
             if timed:
                 enc_ms.append((a, b))
         if do_dec:
             a, b = ev(), ev()
             a.record(stream)
-            q.decode(codes, out=x, stream=stream)
+            q_dec.decode(dcodes, out=x, stream=stream)
             b.record(stream)
             if timed:
                 dec_ms.append((a, b))
@@ -340,7 +397,8 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize(device)
-    assert q.get_error(stream) == 0
+    for q in {id(v): v for v in (q_enc, q_dec) if v is not None}.values():
+        assert q.get_error(stream) == 0
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
@@ -355,7 +413,9 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(device)
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist, device)
-    status = q.get_error(stream)
+    status = 0
+    for q in {id(v): v for v in (q_enc, q_dec) if v is not None}.values():
+        status = status or q.get_error(stream)
     enc_avg = sum(a.elapsed_time(b) for a, b in enc_ms) / max(len(enc_ms), 1)
     dec_avg = sum(a.elapsed_time(b) for a, b in dec_ms) / max(len(dec_ms), 1)
     ms_per_step = elapsed_ms / args.steps
@@ -365,31 +425,39 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         k = max(4, min(args.steps, 10))
-        # two sets of device buffers; the host side holds one input and two result buffers
-        h_codes = [torch.empty((n, n_q), dtype=torch.int16, pin_memory=True) for _ in range(2)]
+        # two sets of device buffers; the host side holds one input set and two result sets
+        h_z = None
+        if do_enc:
+            h_z = torch.empty(z.shape, dtype=z.dtype, pin_memory=True)
+            h_z.copy_(z)
+        h_dc = None
+        if do_dec and not work["decode_own_codes"]:
+            h_dc = torch.empty(dcodes.shape, dtype=dcodes.dtype, pin_memory=True)
+            h_dc.copy_(dcodes)
+        h_codes = ([torch.empty((n, n_q), dtype=torch.int16, pin_memory=True) for _ in range(2)]
+                   if do_enc else None)
         h_x = ([torch.empty((n, 512), dtype=torch.float32, pin_memory=True) for _ in range(2)]
                if do_dec else None)
-        codes2 = [codes, torch.empty_like(codes)]
-        x2 = [x, torch.empty_like(x)] if do_dec else None
-        if do_enc:
-            h_in = torch.empty(z.shape, dtype=z.dtype, pin_memory=True)
-            h_in.copy_(z)
-            in2 = [z, torch.empty_like(z)]
-        else:
-            h_in = torch.empty(codes.shape, dtype=codes.dtype, pin_memory=True)
-            h_in.copy_(codes)
-            in2 = codes2
-        bi = h_in.numel() * h_in.element_size()
+        z2 = [z, torch.empty_like(z)] if do_enc else None
+        codes2 = [codes, torch.empty_like(codes)] if do_enc else None
+        if do_dec:
+            dcodes2 = codes2 if work["decode_own_codes"] else [dcodes, torch.empty_like(dcodes)]
+            x2 = [x, torch.empty_like(x)]
+        bi = ((h_z.numel() * h_z.element_size() if h_z is not None else 0)
+              + (h_dc.numel() * 2 if h_dc is not None else 0))
         bo = (codes.numel() * 2 if do_enc else 0) + (x.numel() * 4 if do_dec else 0)
 
         def h2d(b):
-            in2[b].copy_(h_in, non_blocking=True)
+            if h_z is not None:
+                z2[b].copy_(h_z, non_blocking=True)
+            if h_dc is not None:
+                dcodes2[b].copy_(h_dc, non_blocking=True)
 
         def compute(b, s):
             if do_enc:
-                q.encode(in2[b], n_q=n_q, variant=variant, out=codes2[b], stream=s)
+                q_enc.encode(z2[b], n_q=n_q, variant=variant, out=codes2[b], stream=s)
             if do_dec:
-                q.decode(codes2[b], out=x2[b], stream=s)
+                q_dec.decode(dcodes2[b], out=x2[b], stream=s)
 
         def d2h(b):
             if do_enc:
@@ -412,18 +480,21 @@ def run_ours(args, rank, world, local_rank):
 
     peaks = load_peaks()
     kernels = []
-    lat_bytes = 2048 if work.get("dtype", "f32") == "f32" else 1024
+    lat_dtype = enc["dtype"] if do_enc else None
+    lat_bytes = 2048 if lat_dtype == "f32" else 1024
     if do_enc:
         tf = enc_flop(n_q) * n / (enc_avg / 1e3) / 1e12
         # the captured DRAM traffic is for the full 8-codebook, variant-0 encode
-        tr = (NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + work.get("dtype", "f32"))
+        tr = (NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + lat_dtype)
               if (n_q, variant) == (8, 0) else None)
         kernels.append({
             "kernel": "encode call (k_encode_tc + float32 re-encode)", "bound": "tensor",
-            "achieved": tf, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-            "frac": tf / peaks["bf16_tflops_sustained"],
-            "traffic": tr[0] * n if tr else None, "traffic_source": tr[1] if tr else None,
-            "ms": enc_avg,
+            "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops"],
+            "peak_source": f"{peaks['source']} bf16_tflops (burst: the call is timed alone)",
+            "traffic": tr[0] * n if tr and tr[0] else None,
+            "traffic_source": tr[1] if tr and tr[0] else None,
+            "ms": enc_avg, "frames": n, "latent_dtype": lat_dtype,
             "algorithmic": (f"{enc_flop(n_q)} FLOP/frame x {n} frames; "
                             f"HBM {lat_bytes + 2 * n_q} B/frame"),
             "hbm_gbs": (lat_bytes + 2 * n_q) * n / (enc_avg / 1e3) / 1e9})
@@ -432,23 +503,26 @@ def run_ours(args, rank, world, local_rank):
         tr = NCU_TRAFFIC_PER_UNIT["k_decode"] if n_q == 8 else None
         kernels.append({
             "kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": tr[0] * n if tr else None,
-            "traffic_source": tr[1] if tr else None, "ms": dec_avg,
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "peak_source": f"{peaks['source']} hbm_gbs",
+            "traffic": tr[0] * n if tr and tr[0] else None,
+            "traffic_source": tr[1] if tr and tr[0] else None, "ms": dec_avg, "frames": n,
+            "codes": "from the encode" if work["decode_own_codes"] else
+                     "semantic uniform, acoustic Zipf(1.1)",
             "algorithmic": f"{dec_bytes(n_q)} B/frame x {n} frames (codes in, fp32 latents out)"})
-    dominant = kernels[0]
+    dominant = max(kernels, key=lambda kk: kk["ms"])
     roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roofline["kernel"] = dominant["kernel"]
     roofline["traffic_source"] = dominant.get("traffic_source")
-    roofline["peak_source"] = (f"{peaks['source']} "
-                               f"{'bf16_tflops_sustained' if dominant['bound'] == 'tensor' else 'hbm_gbs'}")
+    roofline["peak_source"] = dominant["peak_source"]
     if args.self_profile and do_enc and (n_q, variant) == (8, 0):
-        _, cyc = q.encode_profile(z, out=codes, stream=stream)
+        _, cyc = q_enc.encode_profile(z, out=codes, stream=stream)
         total = max(cyc["cta_total"], 1)
-        counts = set(q.PROFILE_COUNTS)
+        counts = set(q_enc.PROFILE_COUNTS)
         kernels[0]["self_profile_share"] = {k: round(v / total, 4) for k, v in cyc.items()
                                             if k not in counts}
-        kernels[0]["self_profile_counts"] = {k: cyc[k] for k in q.PROFILE_COUNTS}
-    launches_per_step = (2 if do_enc else 0) + (1 if do_dec else 0)
+        kernels[0]["self_profile_counts"] = {k: cyc[k] for k in q_enc.PROFILE_COUNTS}
+    launches_per_step = (ENCODE_LAUNCHES if do_enc else 0) + (1 if do_dec else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -456,8 +530,8 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16 products, f32 accumulate/re-score", "data": "synthetic",
         "config": {"workload": f"{name}: {WORKLOADS[name]}" + (
                        f" (reduced to {n} frames)" if args.frames else ""), "frames_per_gpu": n,
-                   "latent_dtype": work.get("dtype"), "n_q": n_q, "variant": variant,
-                   "parallelism": f"replicas x{world}",
+                   "halves": _halves(work), "latent_dtype": lat_dtype, "n_q": n_q,
+                   "variant": variant, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (not re-read from L2 between steps)"},
         "realtime_streams": value / FRAME_HZ,
         "roofline": roofline, "kernels": kernels,
@@ -465,7 +539,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(), "status": status, "e2e": e2e,
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(work, name, n_q=n_q, variant=variant)
+        line["cpu_baseline"] = cpu_baseline(work, n_q=n_q, variant=variant)
     if dist:
         dist.destroy_process_group()
     return line
@@ -675,7 +749,8 @@ def run_reference(args):
         work = {"frames": len(text_h)}
     elif name == "streaming":
         model, frames = synth.streaming_step(1024, calls=1)
-        work = {"model": model, "z": frames[0], "frames": frames.shape[1]}
+        work = {"enc": {"model": model, "z": frames[0], "dtype": "f32"}, "dec": None,
+                "frames": frames.shape[1], "decode_own_codes": False}
     else:
         work = make_workload(name, 0)
 
@@ -684,14 +759,7 @@ def run_reference(args):
             oracle.embed_sum(tables_h, rows,
                              oracle.delay_pack(text_h[:nf], audio_h[:, :nf], MOSHI_DELAYS))
             return
-        m = work["model"]
-        if name in ("offline_batch", "bulk_tokenization", "streaming"):
-            c, _, _ = oracle.encode(work["z"][:nf], m.W_in, m.C, n_q=args.n_q,
-                                    variant=args.variant)
-            if name == "offline_batch":
-                oracle.decode(c, m.C, m.W_out)
-        else:
-            oracle.decode(np.ascontiguousarray(work["codes"][:nf, :args.n_q]), m.C, m.W_out)
+        oracle_step(work, nf, args.n_q, args.variant)
 
     t0 = time.perf_counter()
     one(32)
@@ -706,27 +774,60 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     value = nf / dt
     cores = oracle.threads(0)
-    sample = f"first {nf} frames of {name} per step, float64 oracle"
+    what = "pack + embedding sum" if name == "moshi_input" else _halves(work)
+    sample = f"first {nf} frames of {name} per step ({what}), float64 oracle"
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "frames/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{name}: {WORKLOADS[name]}", "sample_frames": nf,
                        **({"n_q": args.n_q, "variant": args.variant}
-                          if name in ("offline_batch", "bulk_tokenization", "decode_heavy")
-                          else {})},
+                          if name not in ("moshi_input", "streaming") else {})},
             "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
+# --------------------------------------------------------------------- launch
+
+
+def check_world(gpus, env):
+    """How this process runs --gpus N: "run" when it is one rank of a world of N processes
+    (torchrun sets WORLD_SIZE) or N = 1 without torchrun; "launch" when N > 1 and no torchrun
+    environment is present, so the script must start the N ranks itself. A world size that
+    differs from N is an error (SystemExit), never a silent single replica."""
+    if gpus < 1:
+        raise SystemExit(f"bench.py: --gpus must be >= 1 (got {gpus})")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise SystemExit(f"bench.py: --gpus {gpus} but this world has WORLD_SIZE={world} "
+                             f"processes; launch N processes for --gpus N")
+        return "run"
+    return "launch" if gpus > 1 else "run"
+
+
+def torchrun_command(argv, gpus, port):
+    """The command that runs this script as `gpus` ranks on one node (127.0.0.1 rendezvous)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__), *argv]
+
+
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="offline_batch", choices=list(WORKLOADS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="encode_decode_1m", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--calls", type=int, default=1000, help="streaming workload: calls per B")
     ap.add_argument("--frames", type=int, default=None,
@@ -743,6 +844,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+
+    if check_world(args.gpus, os.environ) == "launch":
+        sys.exit(subprocess.call(torchrun_command(sys.argv[1:], args.gpus, free_port())))
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

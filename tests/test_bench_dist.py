@@ -26,7 +26,7 @@ def _rank(rank, world, port, out):
     dist = bench.init_dist(world, backend="gloo")
     slowest = bench.max_over_ranks(1.5 * (rank + 1), dist, "cpu")
     work = bench.make_workload("offline_batch", rank, frames=4)
-    row = torch.from_numpy(work["z"][0, :8].copy())
+    row = torch.from_numpy(work["enc"]["z"][0, :8].copy())
     rows = [torch.empty_like(row) for _ in range(world)]
     dist.all_gather(rows, row)
     rate = bench.whole_job_rate(work["frames"], world, slowest)
@@ -57,7 +57,7 @@ def test_two_gloo_ranks():
 def test_reference_arm_runs_on_rank_zero_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
 
@@ -82,3 +82,41 @@ def test_bench_options():
     assert out.returncode == 0 and "--n-q" in out.stdout and "--variant" in out.stdout
     assert run("--n-q", "9").returncode != 0
     assert run("--variant", "2").returncode != 0
+
+
+def test_world_size_must_match_gpus():
+    """--gpus N is never a silent single replica: under torchrun the world must have N ranks;
+    without torchrun and N > 1 the script starts the N ranks itself (on 127.0.0.1)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.check_world(1, {}) == "run"
+    assert bench.check_world(8, {}) == "launch"
+    assert bench.check_world(4, {"WORLD_SIZE": "4"}) == "run"
+    with pytest.raises(SystemExit):
+        bench.check_world(8, {"WORLD_SIZE": "1"})
+    with pytest.raises(SystemExit):
+        bench.check_world(0, {})
+    cmd = bench.torchrun_command(["--gpus", "4", "--steps", "3"], 4, 29500)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"] and cmd[-5].endswith("bench.py")
+    # a mismatched world exits non-zero before any work
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4",
+                        "--impl", "reference", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE=2" in r.stderr
+
+
+def test_two_part_workload_is_built_from_both_configs():
+    """The default step pairs the 1M-frame bf16 encode with the 1M-frame decode-heavy codes,
+    each on its own seeded model (shrunk here)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    w = bench.make_workload("encode_decode_1m", 0, frames=16)
+    assert w["enc"]["dtype"] == "bf16" and w["enc"]["z"].shape == (16, 512)
+    assert w["dec"]["codes"].shape == (16, 8) and not w["decode_own_codes"]
+    assert not (w["enc"]["model"].C == w["dec"]["model"].C).all()
+    off = bench.make_workload("offline_batch", 0, frames=16)
+    assert off["dec"] is None and off["decode_own_codes"]
+    assert bench.make_workload("decode_heavy", 0, frames=16)["enc"] is None
