@@ -215,10 +215,15 @@ int mimi_rvq_stats(mimi_rvq_t h, struct CUstream_st *stream, int64_t *frames_enc
  * exact float32 scores, slow). Its one piece of scratch, the squared codeword
  * norms, lives in a 64 KiB static device array (at most 8 codebooks of 2048;
  * n_q outside 1..8 returns MIMI_RVQ_EINVAL) that every GPU loading the
- * library holds until exit. The first call on a device looks up that array's
- * address; make it before any stream capture. Every call shares the array and
- * rewrites it, so calls that overlap on the GPU (other streams, other host
- * threads) race: serialise them.
+ * library holds until exit. The first call in a CUDA context on a device
+ * looks up that array's address (again after a device reset, which loads the
+ * library's module into a new context); make that first call before any
+ * stream capture. Every call shares the array and rewrites it, so calls that
+ * overlap on the GPU (other streams, other host threads) race: serialise them.
+ * Alignment (this call only; the 16-byte rule of the other calls does not
+ * apply): codebooks 16 bytes (read as float4), W_in 4 bytes, latents 4 bytes
+ * for MIMI_RVQ_F32 and 2 bytes for MIMI_RVQ_BF16, codes 2 bytes; otherwise
+ * MIMI_RVQ_EINVAL.
  */
 int mimi_rvq_encode_noalloc(const float *codebooks, const float *W_in, const void *latents,
                             int dtype, int64_t N, int n_q, int16_t *codes,

@@ -77,10 +77,33 @@ int mimi_rvq_delay_unpack(const int32_t *packed, int64_t S, int K, int col0,
  * A negative token is an absent stream and adds nothing; a token >= rows[k]
  * adds nothing and is counted into *n_bad (device uint64, caller-zeroed; may
  * be NULL).
+ * Failure: the bf16, d = 4096 form waits on its copies with bounded waits
+ * (about 2 s). If one runs out, the kernel stops, lets the copies it issued
+ * land, and returns early (the output is then undefined); it records the
+ * timeout in the library's token-stream status word, which
+ * mimi_rvq_streams_get_error() reports, and also sets *n_bad to UINT64_MAX
+ * when n_bad is not NULL.
  */
 int mimi_rvq_embed_sum(const void *tables, int table_dtype, int K, const int64_t *rows, int d,
                        const int32_t *tokens, int64_t S, void *out, int out_dtype,
                        uint64_t *n_bad, struct CUstream_st *stream);
+
+/*
+ * Status of the token-stream kernels since the last call: synchronises
+ * `stream`, then returns and clears the status word that a timed-out wait of
+ * mimi_rvq_embed_sum sets (MIMI_RVQ_ETIMEOUT; MIMI_RVQ_OK if none; ECUDA if a
+ * CUDA call fails). The word is shared by every caller in the process.
+ */
+int mimi_rvq_streams_get_error(struct CUstream_st *stream);
+
+/*
+ * Failure-path self-test of mimi_rvq_embed_sum's bounded waits, without
+ * hanging or faulting the GPU: launches the embedding-sum kernel in a form
+ * whose producers issue no copy, so its consumers' wait runs out a short
+ * budget (about 50 ms); the kernel records the timeout and returns, and the
+ * next mimi_rvq_streams_get_error returns MIMI_RVQ_ETIMEOUT. Needs no buffers.
+ */
+int mimi_rvq_streams_wait_selftest(struct CUstream_st *stream);
 
 #ifdef __cplusplus
 }

@@ -23,7 +23,9 @@ EXPORTS = ("mimi_rvq_create", "mimi_rvq_destroy", "mimi_rvq_encode", "mimi_rvq_e
            "mimi_rvq_encode_step", "mimi_rvq_project", "mimi_rvq_encode_scan", "mimi_rvq_decode",
            "mimi_rvq_decode_ex", "mimi_rvq_get_error", "mimi_rvq_stats", "mimi_rvq_strerror",
            "mimi_rvq_encode_profile", "mimi_rvq_delay_pack", "mimi_rvq_delay_unpack",
-           "mimi_rvq_embed_sum", "mimi_rvq_wait_selftest", "mimi_rvq_encode_step_ex")
+           "mimi_rvq_embed_sum", "mimi_rvq_wait_selftest", "mimi_rvq_encode_step_ex",
+           "mimi_rvq_encode_noalloc", "mimi_rvq_streams_get_error",
+           "mimi_rvq_streams_wait_selftest")
 TEXT_CARD, TEXT_PAD, AUDIO_PAD = 32000, 32000, 2048
 
 _lib = None
@@ -81,6 +83,10 @@ def library() -> ctypes.CDLL:
     lib.mimi_rvq_delay_unpack.restype = ci
     lib.mimi_rvq_embed_sum.argtypes = [vp, ci, ci, vp, ci, vp, i64, vp, ci, vp, vp]
     lib.mimi_rvq_embed_sum.restype = ci
+    lib.mimi_rvq_streams_get_error.argtypes = [vp]
+    lib.mimi_rvq_streams_get_error.restype = ci
+    lib.mimi_rvq_streams_wait_selftest.argtypes = [vp]
+    lib.mimi_rvq_streams_wait_selftest.restype = ci
     _lib = lib
     return lib
 
@@ -318,3 +324,16 @@ def embed_sum(tables, rows, tokens, out_dtype=None, out=None, n_bad=None, stream
                                         None if n_bad is None else n_bad.data_ptr(),
                                         _stream(stream)), "mimi_rvq_embed_sum")
     return out
+
+
+def streams_get_error(stream=None) -> int:
+    """Synchronise the stream; return and clear the token-stream status word (0 = ok, -6 =
+    a wait of embed_sum timed out)."""
+    return int(library().mimi_rvq_streams_get_error(_stream(stream)))
+
+
+def streams_wait_selftest(stream=None):
+    """Launch the embedding-sum kernel in its self-test form: its wait never completes and
+    times out after ~50 ms; the next streams_get_error() returns -6."""
+    _check(library().mimi_rvq_streams_wait_selftest(_stream(stream)),
+           "mimi_rvq_streams_wait_selftest")

@@ -22,8 +22,8 @@ def sources():
 
 
 def inputs():
-    return sources() + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + [
-        os.path.join(ROOT, "include", "mimi_rvq.h")]
+    return (sources() + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")))
+            + sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
 
 
 def up_to_date() -> bool:

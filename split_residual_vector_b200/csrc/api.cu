@@ -80,7 +80,9 @@ void free_tables(mimi::Tables& t) {
                     t.wide_bars, t.wide_partial};
     for (void* p : ptrs)
         if (p) cudaFree(p);
+    const int sms = t.num_sms;
     t = mimi::Tables{};
+    t.num_sms = sms;
 }
 
 template <class T>
@@ -141,6 +143,7 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     h->device = dev;
     h->num_sms = prop.multiProcessorCount;
     mimi::Tables& t = h->t;
+    t.num_sms = h->num_sms;
     const size_t nC = (size_t)kQ * kK * kD;
     cudaError_t e = cudaSuccess;
     if (e == cudaSuccess) e = dalloc(&t.C32, nC);

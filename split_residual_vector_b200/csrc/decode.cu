@@ -61,7 +61,7 @@ cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int 
                           cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
     int64_t blocks = (n + kWarps - 1) / kWarps;
-    const int64_t cap = 148 * 8;  // 8 resident blocks of 8 warps per SM
+    const int64_t cap = (int64_t)t.num_sms * 8;  // 8 resident blocks of 8 warps per SM
     if (blocks > cap) blocks = cap;
     k_decode<<<(int)blocks, kWarps * 32, 0, s>>>(t.P, codes, n, n_q, out, t.err);
     return cudaGetLastError();

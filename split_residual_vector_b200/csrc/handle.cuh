@@ -30,6 +30,7 @@ constexpr int kWideMaxGroups = 64;    // group barriers (the last one is the wai
 constexpr int kWideBarStride = 32;    // words per group barrier (count, generation; own 128 B line)
 
 struct Tables {
+    int num_sms = 148;            // SMs of the handle's device (grid sizes)
     // float32 originals
     float* C32 = nullptr;         // [Q][K][D] codebooks (0 semantic)
     float* Win32 = nullptr;       // [D][Din] W_in

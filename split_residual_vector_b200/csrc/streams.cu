@@ -21,9 +21,17 @@
 
 #include <cstdint>
 
+#include "../../include/mimi_rvq.h"
 #include "../../include/mimi_rvq_streams.h"
+#include "ptx.cuh"
 
 namespace mimi {
+
+// Error bits (MIMI_DEV_ERR_*) of the handle-free token-stream calls: a kernel
+// whose bounded wait ran out sets MIMI_DEV_ERR_TIMEOUT here, whether or not the
+// caller passed an n_bad counter; mimi_rvq_streams_get_error reads and clears it.
+static __device__ int g_stream_err;
+
 namespace {
 
 constexpr int kQ = 8;
@@ -285,9 +293,10 @@ __device__ __forceinline__ void bar_arrive_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 // Bounded wait for the phase of the given parity; false if the budget ran out
-// or another thread of the CTA already gave up (*stop != 0; the caller then
-// records the failure in *stop).
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* stop) {
+// or another thread of the CTA already gave up (*stop != 0, unless stop is
+// null; the caller then records the failure in *stop).
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* stop,
+                                         long long budget) {
     const long long t0 = clock64();
     while (true) {
         uint32_t ok;
@@ -299,7 +308,7 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatil
             : "r"(smem_addr(bar)), "r"(parity)
             : "memory");
         if (ok) return true;
-        if (*stop || clock64() - t0 > kSpinBudget) return false;
+        if ((stop != nullptr && *stop) || clock64() - t0 > budget) return false;
     }
 }
 __device__ __forceinline__ void bulk_copy(void* smem_dst, const void* src, uint32_t bytes,
@@ -320,17 +329,22 @@ __device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t x) {
         : "r"(x));
 }
 
-template <int NST, typename OT, int D>
+// kSelfTest: the instantiation of the wait self-test. Its producers issue no
+// copy and never arrive, so the consumers' first wait runs out its (short)
+// budget and the failure path below runs; it reads no tokens or tables and
+// stores nothing.
+template <int NST, typename OT, int D, bool kSelfTest = false>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     k_embed_sum_tma(const __nv_bfloat16* __restrict__ tables, Tables tb, int K,
                     const int32_t* __restrict__ tokens, int64_t S, OT* __restrict__ out,
-                    unsigned long long* __restrict__ n_bad) {
+                    unsigned long long* __restrict__ n_bad, long long budget) {
     constexpr int d = D;
     constexpr int G = kGroupBytes / (2 * D) < 32 ? kGroupBytes / (2 * D) : 32;  // rows per stage
     static_assert(G >= 1 && D % 8 == 0 && D <= kConsumerWarps * 32 * 8, "shape");
     extern __shared__ __align__(128) uint8_t ring[];  // [NST][G][D] bf16
     __shared__ __align__(8) uint64_t full[NST], empty[NST];
     __shared__ uint32_t valid[NST];
+    __shared__ int64_t last_issued[kProducerWarps];   // last stage each producer copied
     __shared__ volatile int failed;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int groups = (K + G - 1) / G;
@@ -341,16 +355,19 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         for (int b = 0; b < NST; ++b) {
             bar_init(&full[b], 1);
             bar_init(&empty[b], kConsumerWarps);
+            valid[b] = 0;
         }
+        for (int p = 0; p < kProducerWarps; ++p) last_issued[p] = -1;
         failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
     if (warp >= kConsumerWarps) {
-        // ---- producer warps: warp p takes stages j = p, p + P, ...
+        // ---- producer warps: warp p takes stages j = p, p + P, ...; none once a wait failed
         const int p = warp - kConsumerWarps;
-        for (int64_t j = p; j < n_stages; j += kProducerWarps) {
+        for (int64_t j = p; j < n_stages && !kSelfTest; j += kProducerWarps) {
+            if (failed) break;
             const int b = (int)(j % NST);
             const int g = (int)(j % groups);
             const int64_t s = blockIdx.x + (j / groups) * gridDim.x;
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             const uint32_t mask = __ballot_sync(0xffffffffu, ok);
             if (j >= NST) {  // wait until the consumers released this buffer
                 int w = 1;
-                if (lane == 0) w = bar_wait(&empty[b], (uint32_t)((j / NST - 1) & 1), &failed);
+                if (lane == 0) w = bar_wait(&empty[b], (uint32_t)((j / NST - 1) & 1), &failed, budget);
                 if (!__shfl_sync(0xffffffffu, w, 0)) {
                     if (lane == 0) failed = 1;
                     break;
@@ -373,6 +390,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             }
             if (lane == 0) {
                 valid[b] = mask;
+                last_issued[p] = j;
                 bar_arrive_tx(&full[b], (uint32_t)__popc(mask) * row_bytes);
             }
             __syncwarp();
@@ -391,7 +409,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[e] = 0.f;
             // after a failed wait the thread stops waiting but the loop runs on
-            if (!failed && !bar_wait(&full[b], (uint32_t)((j / NST) & 1), &failed)) failed = 1;
+            const bool have = !failed && bar_wait(&full[b], (uint32_t)((j / NST) & 1), &failed, budget);
+            if (!have) failed = 1;
             const uint32_t mask = valid[b];
             if (c8 < d) {
                 const uint8_t* buf = ring + b * stage_bytes + c8 * 2;
@@ -408,16 +427,31 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
                         add_bf16x2(acc[6], acc[7], w[i].w);
                     }
             }
-            __syncwarp();
-            if (lane == 0) bar_arrive(&empty[b]);
-            if (g == groups - 1 && c8 < d) {
+            // a buffer is released only by warps whose every lane saw its copies land, so
+            // after a failure no copy is issued into a buffer that may still be filling
+            if (__all_sync(0xffffffffu, have) && lane == 0) bar_arrive(&empty[b]);
+            if (!kSelfTest && g == groups - 1 && c8 < d) {
                 const int64_t s = blockIdx.x + (j / groups) * gridDim.x;
                 store8(out + s * d + c8, acc);
             }
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0 && failed && n_bad != nullptr) atomicExch(n_bad, ~0ull);
+    if (threadIdx.x == 0 && failed) {
+        atomicOr(&g_stream_err, MIMI_DEV_ERR_TIMEOUT);
+        if (n_bad != nullptr) atomicExch(n_bad, ~0ull);
+        // Copies already issued may still be landing in the ring; each buffer has at most
+        // one (a buffer is refilled only after its previous copies landed), the last stage
+        // issued into it. Wait for each of those (bounded) before the CTA exits.
+        for (int b = 0; b < NST; ++b) {
+            int64_t jl = -1;
+            for (int p = 0; p < kProducerWarps; ++p)
+                for (int64_t j = last_issued[p]; j >= 0 && j > last_issued[p] - (int64_t)kProducerWarps * NST;
+                     j -= kProducerWarps)
+                    if (j % NST == b && j > jl) jl = j;
+            if (jl >= 0) bar_wait(&full[b], (uint32_t)((jl / NST) & 1), nullptr, budget);
+        }
+    }
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -516,7 +550,8 @@ cudaError_t launch_embed_tma_n(const void* tables, const Tables& tb, int K, int 
     const int grid = (int)(S < sms ? S : sms);
     (void)d;
     k_embed_sum_tma<NST, OT, D><<<grid, kTmaThreads, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(tables), tb, K, tokens, S, static_cast<OT*>(out), n_bad);
+        static_cast<const __nv_bfloat16*>(tables), tb, K, tokens, S, static_cast<OT*>(out), n_bad,
+        kSpinBudget);
     return cudaGetLastError();
 }
 
@@ -552,8 +587,40 @@ cudaError_t launch_embed(const void* tables, const Tables& tb, int K, int d, con
     return cudaGetLastError();
 }
 
+// ~50 ms at 2 GHz: long enough to be a real wait, short for a test.
+constexpr long long kSelftestBudget = 100000000LL;
+
+cudaError_t launch_embed_selftest(cudaStream_t s) {
+    auto* k = k_embed_sum_tma<2, __nv_bfloat16, kTmaWidth, true>;
+    const int smem = 2 * tma_group(kTmaWidth) * kTmaWidth * 2;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    Tables tb{};
+    k<<<1, kTmaThreads, smem, s>>>(nullptr, tb, MIMI_RVQ_MAX_STREAMS / 4, nullptr, 1, nullptr,
+                                   nullptr, kSelftestBudget);
+    return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace mimi
+
+extern "C" int mimi_rvq_streams_get_error(struct CUstream_st* stream) {
+    using namespace mimi;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return status(cudaErrorUnknown);
+    int bits = 0;
+    if (cudaMemcpyFromSymbol(&bits, g_stream_err, sizeof(int)) != cudaSuccess)
+        return status(cudaErrorUnknown);
+    if (bits) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_stream_err, &zero, sizeof(int)) != cudaSuccess)
+            return status(cudaErrorUnknown);
+    }
+    return (bits & MIMI_DEV_ERR_TIMEOUT) ? MIMI_RVQ_ETIMEOUT : MIMI_RVQ_OK;
+}
+
+extern "C" int mimi_rvq_streams_wait_selftest(struct CUstream_st* stream) {
+    return mimi::status(mimi::launch_embed_selftest(stream));
+}
 
 extern "C" int mimi_rvq_delay_pack(const int32_t* text, const int16_t* audio, int n_audio,
                                    int64_t T, const int32_t* delays, int64_t S, int32_t text_pad,

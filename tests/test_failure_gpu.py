@@ -33,3 +33,25 @@ def test_a_wait_that_never_completes_times_out_and_the_handle_recovers(which):
     assert q.get_error() == 0
     with pytest.raises(pkg.MimiRVQError):
         q.wait_selftest(2)
+
+
+def test_embedding_sum_wait_times_out_reports_and_recovers():
+    """The embedding sum's bulk-copy wait, in its self-test form (no copy is ever issued):
+    the consumers' wait runs out, the kernel records the timeout in the token-stream status
+    word (no n_bad counter is involved), returns, and the next real call is exact."""
+    import oracle
+    import split_residual_vector_b200 as pkg
+    rows = synth.moshi_rows()
+    tables = synth.moshi_tables(seed=21)
+    text, audio = synth.moshi_streams(40, seed=22)
+    V = oracle.delay_pack(text, audio, [0, 1, 1, 1, 1, 1, 1, 1])
+    tt = torch.from_numpy(tables.view(np.int16)).cuda().view(torch.bfloat16)
+    tok = torch.from_numpy(np.ascontiguousarray(V)).cuda()
+    before = pkg.embed_sum(tt, rows, tok, out_dtype=torch.float32).cpu().numpy()
+    assert pkg.streams_get_error() == 0
+    pkg.streams_wait_selftest()
+    assert pkg.streams_get_error() == ETIMEOUT   # reported once ...
+    assert pkg.streams_get_error() == 0          # ... and cleared
+    after = pkg.embed_sum(tt, rows, tok, out_dtype=torch.float32).cpu().numpy()
+    assert pkg.streams_get_error() == 0
+    assert np.array_equal(after, before)
