@@ -222,7 +222,8 @@ class Quantizer:
     PROFILE_SLOTS = ("producer_wait_stage", "mma_wait_operands", "mma_wait_score_buffer",
                      "mma_wait_level_operand", "mma_wait_latents", "epi_wait_score_tile",
                      "epi_scan", "epi_pick", "epi_update", "epi_stage", "epi_barrier",
-                     "cta_total", "n_chunks", "n_displaced", "n_runner_up", "n_more")
+                     "cta_total", "n_chunks", "n_displaced", "n_runner_up", "n_more",
+                     "pick_exchange_merge", "pick_rescore", "pick_select", "scan_drain")
     PROFILE_COUNTS = ("n_chunks", "n_displaced", "n_runner_up", "n_more")
 
     def encode_profile(self, latents, out=None, stream=None):
@@ -231,7 +232,7 @@ class Quantizer:
         import torch
         n, dt = self._latents(latents)
         out = self._codes_out(n, out)
-        cyc = torch.zeros(16, dtype=torch.int64, device=self.device)
+        cyc = torch.zeros(len(self.PROFILE_SLOTS), dtype=torch.int64, device=self.device)
         _check(library().mimi_rvq_encode_profile(self._h, latents.data_ptr(), dt, n,
                                                  out.data_ptr(), cyc.data_ptr(), _stream(stream)),
                "mimi_rvq_encode_profile")

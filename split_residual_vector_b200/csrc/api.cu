@@ -60,14 +60,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x 128 rows,
-// 128-byte swizzle: the layout the UMMA shared-memory descriptors expect.
+// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x 256 rows
+// (32 KiB: one stage of the tensor-core encoder's ring), 128-byte swizzle: the
+// layout the UMMA shared-memory descriptors expect.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, 256};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -75,7 +76,7 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 }
 
 void free_tables(mimi::Tables& t) {
-    void* ptrs[] = {t.C32, t.Win32, t.WinT32, t.Cbf, t.Win_hi, t.Win_lo, t.cnorm, t.cbound,
+    void* ptrs[] = {t.C32, t.Win32, t.WinT32, t.Cbf, t.Win_hi, t.Win_lo, t.cnorm, t.cnorm3, t.cbound,
                     t.P, t.err, t.rescan_count, t.rescan_list, t.stats, t.wide_y,
                     t.wide_bars, t.wide_partial};
     for (void* p : ptrs)
@@ -153,6 +154,7 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (e == cudaSuccess) e = dalloc(&t.Win_hi, (size_t)kD * kDin);
     if (e == cudaSuccess) e = dalloc(&t.Win_lo, (size_t)kD * kDin);
     if (e == cudaSuccess) e = dalloc(&t.cnorm, (size_t)kQ * kK);
+    if (e == cudaSuccess) e = dalloc(&t.cnorm3, (size_t)kQ * kK * 4);
     if (e == cudaSuccess) e = dalloc(&t.cbound, (size_t)4 * kQ);
     if (e == cudaSuccess) e = dalloc(&t.P, (size_t)kQ * kK * kDin);
     if (e == cudaSuccess) e = dalloc(&t.err, 1);

@@ -61,7 +61,9 @@ cudaError_t launch_decode(const Tables& t, const int16_t* codes, int64_t n, int 
                           cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
     int64_t blocks = (n + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)t.num_sms * 8;  // 8 resident blocks of 8 warps per SM
+    // 4 blocks of 8 warps per SM: measured 2 % faster than 8 (0.720 against 0.735 ms
+    // for 1 048 576 frames), 16 was slower (0.78 ms)
+    const int64_t cap = (int64_t)t.num_sms * 4;
     if (blocks > cap) blocks = cap;
     k_decode<<<(int)blocks, kWarps * 32, 0, s>>>(t.P, codes, n, n_q, out, t.err);
     return cudaGetLastError();

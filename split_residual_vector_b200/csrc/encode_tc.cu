@@ -9,11 +9,15 @@
 //      columns [0, 256). Those columns then hold the residual r (float32) for
 //      the whole level chain: it never leaves the SM.
 //   2. for each codebook l = 0 (semantic, on y) and 1..7 (acoustic, on r):
-//      candidate scores ||c||^2 - 2 bf16(r) . bf16(c) for all 2048 codewords
-//      as 16 tcgen05 GEMM tiles [128 x 256] x [256 x 128] (codebook tiles
-//      streamed by TMA into a shared-memory ring; accumulators double-buffered
-//      in TMEM columns [256, 512)). The epilogue keeps a sorted list of the
-//      best 8 candidate keys per row.
+//      candidate half-scores ||c||^2 / 2 - bf16(r) . bf16(c) for all 2048
+//      codewords as 8 tcgen05 GEMM tiles [128 x 256] x [256 x 256]. Each tile
+//      starts with one K = 16 step that writes ||c||^2 / 2 into the accumulator
+//      (A = ones, B = the norm's three exact bf16 parts) and continues with A =
+//      -bf16(r), so the epilogue reads the half-score directly (codebook tiles
+//      streamed by TMA into a shared-memory ring, one 256-row box per stage;
+//      the accumulator is TMEM columns [256, 512), which the epilogue copies
+//      into registers at once so that the next tile's MMAs overlap its scan).
+//      The epilogue keeps a sorted list of the best 8 candidate keys per row.
 //   3. certified pick: with E a rigorous bound on |bf16 score - exact score|
 //      (from ||r||, this row's bf16 rounding residual ||bf16(r) - r||, and the
 //      codebook's max ||c|| and max ||bf16(c) - c||), every codeword outside
@@ -41,14 +45,17 @@ namespace mimi {
 namespace {
 
 constexpr int BM = 128;                 // frames per tile = TMEM lanes
-constexpr int BN = 128;                 // codewords per score tile
+constexpr int BN = 256;                 // codewords per score tile (one N = 256 MMA)
 constexpr int BK = 64;                  // K elements per stage (128 B of bf16)
-constexpr int NT = kK / BN;             // 16 score tiles per codebook
+constexpr int NT = kK / BN;             // 8 score tiles per codebook
 constexpr int KCH = kD / BK;            // 4 K chunks per score tile
 constexpr int PKCH = kDin / BK;         // 8 K chunks of the projection
-constexpr int STAGES = 8;
+// A bulk tensor copy costs the SM about the same time whatever its size (up to
+// a 32 KiB box), so each stage is one 256-row box: a whole score tile's 64-wide
+// K chunk, or every output row of the projection's.
+constexpr int STAGES = 4;
 constexpr int TOPK = 8;                 // candidate list length per row and half
-constexpr int STAGE_BYTES = BN * BK * 2;        // 16 KiB
+constexpr int STAGE_BYTES = BN * BK * 2;        // 32 KiB
 constexpr int A_CHUNK_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int RING_OFF = 0;
 constexpr int A_OFF = STAGES * STAGE_BYTES;             // 128 KiB
@@ -56,13 +63,28 @@ constexpr int X_OFF = A_OFF + KCH * A_CHUNK_BYTES;      // 192 KiB: epilogue exc
 constexpr int XKEYS_OFF = X_OFF;                        // [2][BM][TOPK + 2] keys, best, evicted
 constexpr int XDOT_OFF = XKEYS_OFF + 2 * BM * 10 * 4;   // [2][BM][TOPK] partial re-score dots
 constexpr int XNORM_OFF = XDOT_OFF + 2 * BM * TOPK * 4; // [2][BM][2] partial norms
-constexpr int CN_OFF = XNORM_OFF + 2 * BM * 2 * 4;      // [K] ||c||^2 of the level being scanned
-constexpr int BAR_OFF = CN_OFF + kK * 4;
+// The norm step's operands (16 K elements, no swizzle): B holds the three bf16
+// parts of ||c||^2 / 2 of the score tile's codewords, A holds ones.
+constexpr int NORMB_OFF = XNORM_OFF + 2 * BM * 2 * 4;  // [BN][16] bf16
+constexpr int ONESA_OFF = NORMB_OFF + BN * 32;         // [BM][16] bf16
+constexpr int BAR_OFF = ONESA_OFF + BM * 32;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;        // barriers, slack for 1 KiB alignment
 constexpr int kEpiWarps = 8;            // two per TMEM lane quarter: column halves
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kCtrlWarps = 4;           // warpgroup 0: TMA (warp 0), MMA (warp 1), two idle
+constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384: three warpgroups
+// Registers. The CTA is launched with kLaunchRegs per thread (the most 384
+// threads may have); warpgroup 0 then gives registers back and the two epilogue
+// warpgroups take them (setmaxnreg), since the epilogue holds a whole score
+// tile's half-rows in registers. The split must fit what the CTA was launched
+// with, or the increase would wait forever; the host checks the compiled
+// register count against it before every launch.
+constexpr int kLaunchRegs = 168;
+constexpr int kCtrlRegs = 64;
+constexpr int kEpiRegs = 216;
+static_assert(32 * (kCtrlWarps * kCtrlRegs + kEpiWarps * kEpiRegs) <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_SCORE = 256;    // first score buffer column
+constexpr uint32_t TMEM_SCORE = 256;    // the score buffer: columns [256, 512)
 
 // Candidate bound. With e_r = bf16(r) - r and e_c = bf16(c) - c,
 //   bf16(r).bf16(c) - r.c = r.e_c + e_r.c + e_r.e_c,
@@ -107,17 +129,21 @@ enum ProfSlot {
     P_EPI_ESYNC,        // epilogue barrier waits
     P_CTA_TOTAL,        // whole CTA
     P_N_CHUNK,          // event counts, summed over epilogue warps: 32-column chunks scanned,
-    P_N_DEM,            //   chunks where some lane's displaced best entered the list,
+    P_N_DEM,            //   256-column tiles where some lane put a displaced best in the list,
     P_N_SECOND,         //   chunks where some lane had a runner-up near the window,
     P_N_MORE,           //   chunks where some lane had three or more keys near it
-    kProfSlots = 16
+    P_PICK_XCHG,        // parts of P_EPI_PICK: list exchange (barrier included) and merge,
+    P_PICK_RESCORE,     //   float32 re-score of the window,
+    P_PICK_SELECT,      //   dot exchange (barrier included) and the pick
+    P_SCAN_DRAIN,       // part of P_EPI_SCAN: score tile to registers, next norms, release
+    kProfSlots = 20
 };
 
 struct Bars {
     uint64_t full[STAGES], empty[STAGES];
     uint64_t zfull[2], zempty[2];
     uint64_t yfull, afull, aempty, drain;
-    uint64_t tfull[2], tempty[2];
+    uint64_t tfull, tempty;     // the TMEM score buffer
     uint64_t ebar;          // epilogue-wide barrier (all epilogue threads arrive)
     uint32_t tmem_base;
     int abort;
@@ -202,11 +228,13 @@ __device__ __forceinline__ long long pclock() {
     return 0;
 }
 
+// One CTA per SM (its shared memory and TMEM take the whole SM).
 template <bool kProf>
 __global__ void __launch_bounds__(kThreads, 1)
     k_encode_tc(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_Whi,
                 const __grid_constant__ CUtensorMap tm_Wlo, const float* __restrict__ C32,
-                const float* __restrict__ cnorm, const float* __restrict__ cbound,
+                const float* __restrict__ cnorm, const uint2* __restrict__ cnorm3,
+                const float* __restrict__ cbound,
                 const void* __restrict__ z, int dtype, int64_t n, int n_q, int variant,
                 int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
                 int* rescan_count, int* rescan_list, unsigned long long* stats,
@@ -236,9 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->zfull[b], kEpiWarps);
             mbar_init(&bars->zempty[b], 1);
-            mbar_init(&bars->tfull[b], 1);
-            mbar_init(&bars->tempty[b], kEpiWarps);
         }
+        mbar_init(&bars->tfull, 1);
+        mbar_init(&bars->tempty, kEpiWarps);
         mbar_init(&bars->yfull, 1);
         mbar_init(&bars->afull, kEpiWarps);
         mbar_init(&bars->aempty, 1);
@@ -252,6 +280,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_Whi);
         prefetch_tmap(&tm_Wlo);
     }
+    // the norm step's operands: ones (A, constant) and, for the first score tile
+    // (codebook 0, codewords 0..255), the norms (B); the B tile's second K half is zero
+    for (int i = threadIdx.x; i < BN; i += kThreads) {
+        if (i < BM) {
+            *reinterpret_cast<uint4*>(smem + ONESA_OFF + k16_offset(i, 0)) =
+                make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);  // bf16 1, 1, 1, 0, ...
+            *reinterpret_cast<uint4*>(smem + ONESA_OFF + k16_offset(i, 1)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        const uint2 nv = __ldg(cnorm3 + i);
+        *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(i, 0)) = make_uint4(nv.x, nv.y, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(i, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&bars->tmem_base, TMEM_COLS);
         tmem_relinquish();
@@ -262,7 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
     const long long t_cta0 = pclock<kProf>();
 
-    if (warp == 0) {
+    if (warp < kCtrlWarps) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+      // warps 2 and 3 are idle and wait at the final barrier
+      if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t it = 0;
@@ -281,10 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                for (int kc = 0; kc < PKCH && ok; ++kc) {
-                    ok = ok && load(&tm_Whi, kc * BK, 0) && load(&tm_Whi, kc * BK, BN);
-                    ok = ok && load(&tm_Wlo, kc * BK, 0) && load(&tm_Wlo, kc * BK, BN);
-                }
+                for (int kc = 0; kc < PKCH && ok; ++kc)
+                    ok = ok && load(&tm_Whi, kc * BK, 0) && load(&tm_Wlo, kc * BK, 0);
                 for (int l = 0; l < n_q && ok; ++l)
                     for (int nt = 0; nt < NT && ok; ++nt)
                         for (int kc = 0; kc < KCH && ok; ++kc)
@@ -319,20 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t a_hi = abase + zb * 2 * A_CHUNK_BYTES;
                     const uint32_t a_lo = a_hi + A_CHUNK_BYTES;
-                    for (int g = 0; g < 4 && ok; ++g) {
+                    // g = 0: W_hi (z_hi and z_lo), g = 1: W_lo (z_hi); all 256 outputs at once
+                    for (int g = 0; g < 2 && ok; ++g) {
                         const int s = it % STAGES;
                         ok = twait(&bars->full[s], (it / STAGES) & 1, p_full);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t b = ring + s * STAGE_BYTES;
-                        const uint32_t d = tmem + (g & 1) * BN;
 #pragma unroll
                         for (int k = 0; k < BK / 16; ++k) {
-                            const uint32_t acc = (kc > 0 || k > 0 || g >= 2) ? 1u : 0u;
-                            umma_bf16(d, sw128_desc(a_hi + 32 * k), sw128_desc(b + 32 * k), idesc,
+                            const uint32_t acc = (kc > 0 || k > 0 || g >= 1) ? 1u : 0u;
+                            umma_bf16(tmem, sw128_desc(a_hi + 32 * k), sw128_desc(b + 32 * k), idesc,
                                       acc);
-                            if (g < 2 && f32_in)
-                                umma_bf16(d, sw128_desc(a_lo + 32 * k), sw128_desc(b + 32 * k),
+                            if (g == 0 && f32_in)
+                                umma_bf16(tmem, sw128_desc(a_lo + 32 * k), sw128_desc(b + 32 * k),
                                           idesc, 1u);
                         }
                         umma_commit(&bars->empty[s]);
@@ -351,11 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                     }
                     for (int nt = 0; nt < NT && ok; ++nt) {
-                        const int bsel = tcnt & 1;
-                        ok = twait(&bars->tempty[bsel], ((tcnt >> 1) & 1) ^ 1, p_tempty);
+                        ok = twait(&bars->tempty, (tcnt & 1) ^ 1, p_tempty);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t d = tmem + TMEM_SCORE + bsel * BN;
+                        const uint32_t d = tmem + TMEM_SCORE;
+                        // ||c||^2 / 2 into the accumulator (the epilogue wrote this tile's
+                        // norms before releasing the buffer), then A = -bf16(r)
+                        umma_bf16(d, k16_desc(smem_u32(smem + ONESA_OFF)),
+                                  k16_desc(smem_u32(smem + NORMB_OFF)), idesc, 0u);
                         for (int kc = 0; kc < KCH && ok; ++kc) {
                             const int s = it % STAGES;
                             ok = twait(&bars->full[s], (it / STAGES) & 1, p_full);
@@ -365,12 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t a = abase + kc * A_CHUNK_BYTES;
 #pragma unroll
                             for (int k = 0; k < BK / 16; ++k)
-                                umma_bf16(d, sw128_desc(a + 32 * k), sw128_desc(b + 32 * k), idesc,
-                                          (kc > 0 || k > 0) ? 1u : 0u);
+                                umma_bf16(d, sw128_desc(a + 32 * k), sw128_desc(b + 32 * k), idesc, 1u);
                             umma_commit(&bars->empty[s]);
                             ++it;
                         }
-                        umma_commit(&bars->tfull[bsel]);
+                        umma_commit(&bars->tfull);
                         ++tcnt;
                     }
                     if (updates_after(l) || l == n_q - 1) umma_commit(&bars->aempty);
@@ -386,28 +430,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicAdd(prof + P_MMA_ZFULL, (unsigned long long)p_zfull);
             }
         }
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
         // ------------------------------------------------------------ epilogue
         // Eight warps. Warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows);
-        // the two warps of a lane quarter split every 128-column score tile
-        // (half h takes columns 64 h .. + 63) and the 256 dimensions of r
+        // the two warps of a lane quarter split every 256-column score tile
+        // (half h takes columns 128 h .. + 127) and the 256 dimensions of r
         // (half h owns dimensions 128 h .. + 127). Each thread keeps a sorted
         // list of its half's 8 best keys; the halves merge at the end of a level.
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - kCtrlWarps) >> 2;
         const int row = quarter * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-        float* cn_s = reinterpret_cast<float*>(smem + CN_OFF);
-        const int etid = threadIdx.x - 64;  // 0..255 within the epilogue
-        // copy ||c||^2 of codebook l into shared memory (8 floats per thread); callers
-        // place it after a barrier that ends all reads of the previous level's copy
-        // and before one that precedes the next scan
-        auto stage_cn = [&](int l) {
-            const float4* src = reinterpret_cast<const float4*>(cnorm + (size_t)l * kK);
-            float4* dst = reinterpret_cast<float4*>(cn_s);
-            dst[etid] = __ldg(src + etid);
-            dst[etid + 256] = __ldg(src + etid + 256);
+        const int etid = threadIdx.x - 32 * kCtrlWarps;  // 0..255 within the epilogue: norm-tile row
+        // The score tiles run in the order (frame tile, codebook l, tile nt); after
+        // draining one, thread etid writes its codeword's norm parts for the next into the
+        // norm step's B tile. Each value is loaded one tile ahead of its write.
+        auto next_tile = [&](int& l, int& nt) {
+            if (++nt == NT) {
+                nt = 0;
+                if (++l == n_q) l = 0;
+            }
         };
+        int pf_l = 0, pf_nt = 0;
+        next_tile(pf_l, pf_nt);  // the setup wrote tile (0, 0); this is the one after it
+        uint2 pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
         float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
         float* xdot = reinterpret_cast<float*>(smem + XDOT_OFF);
         float* xnorm = reinterpret_cast<float*>(smem + XNORM_OFF);
@@ -415,6 +463,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         unsigned long long done = 0;
         long long p_tfull = 0, p_scan = 0, p_pick = 0, p_update = 0, p_stage = 0, p_esync = 0;
+        long long p_xchg = 0, p_rescore = 0, p_select = 0, p_drain = 0, t_sub = 0;
+        // attribute the cycles since t_sub to one of the finer counters
+        auto sub = [&](long long& acc) {
+            const long long t = pclock<kProf>();
+            acc += t - t_sub;
+            t_sub = t;
+        };
         unsigned long long n_chunk = 0, n_dem = 0, n_sec = 0, n_more = 0;
         long long t_mark = pclock<kProf>();
         // attribute the cycles since the last mark to one counter
@@ -438,8 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
                 nr2 = fmaf(a, a, nr2);
                 nr2 = fmaf(b, b, nr2);
-                pk[i] = pack_bf16x2(a, b);
-                const float ea = bf16_lo_to_f32(pk[i]) - a, eb = bf16_hi_to_f32(pk[i]) - b;
+                pk[i] = pack_bf16x2(-a, -b);  // the operand is -bf16(r) (rounding is symmetric)
+                const float ea = bf16_lo_to_f32(pk[i]) + a, eb = bf16_hi_to_f32(pk[i]) + b;
                 ner2 = fmaf(ea, ea, ner2);
                 ner2 = fmaf(eb, eb, ner2);
             }
@@ -549,7 +604,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->afull);
-            stage_cn(0);  // visible after the barrier in combine_norms
             ok = combine_norms(nr2, ner2);
             if (!ok) break;
 
@@ -557,89 +611,115 @@ __global__ void __launch_bounds__(kThreads, 1)
             int win_codes[kQ];
             bool flagged = false;
             for (int l = 0; l < n_q && ok; ++l) {
-                const float* cn = cn_s;
                 const float* book = C32 + (size_t)l * kK * kD;
                 const float4 cb = __ldg(reinterpret_cast<const float4*>(cbound) + l);
                 const float cmax = cb.x, cnmax = cb.y, ecmax = cb.z;
                 const float nr = sqrtf(nr2) * 1.0001f, ner = sqrtf(ner2) * 1.0001f;
+                // E bounds |accumulated half-score - exact half-score|: the product error,
+                // the float32 accumulation of the products and of ||c||^2 / 2, and rounding
+                // slack; two keys can each be off by E, hence the window 2 E.
                 const float dot_err = nr * ecmax + ner * cmax + ner * ecmax +
-                                      kAccRel * (nr + ner) * (cmax + ecmax);
-                const float E = 2.f * dot_err * 1.0001f +
-                                kScoreRel * (cnmax + 2.f * (nr + ner) * (cmax + ecmax));
+                                      kAccRel * ((nr + ner) * (cmax + ecmax) + 0.5f * cnmax);
+                const float E = dot_err * 1.0001f +
+                                kScoreRel * (0.5f * cnmax + (nr + ner) * (cmax + ecmax));
                 const float twoE = 2.f * E;
                 Cands cs;
                 cands_reset(cs);
-                // ---- scan this half of the 16 score tiles of the codebook
+                // ---- scan this half of the 8 score tiles of the codebook
                 for (int nt = 0; nt < NT; ++nt) {
-                    const int bsel = tcnt & 1;
                     mark(p_scan);
-                    ok = ewait(&bars->tfull[bsel], (tcnt >> 1) & 1);
+                    ok = ewait(&bars->tfull, tcnt & 1);
                     mark(p_tfull);
                     ++tcnt;
                     if (!ok) break;
                     tc_fence_after();
-                    uint32_t v[2][32];
-                    tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64, v[0]);
-                    tmem_ld32(trow + TMEM_SCORE + bsel * BN + half * 64 + 32, v[1]);
+                    t_sub = pclock<kProf>();
+                    // this half's 128 columns of the tile, all in registers: the buffer is
+                    // released before the scan so that the next tile's MMAs run meanwhile
+                    uint32_t v[4][32];
+#pragma unroll
+                    for (int c2 = 0; c2 < 4; ++c2)
+                        tmem_ld32(trow + TMEM_SCORE + half * 128 + c2 * 32, v[c2]);
                     tmem_wait_ld();
+                    // the norm step of this tile has completed: write the next tile's norms
+                    *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(etid, 0)) =
+                        make_uint4(pf_norm.x, pf_norm.y, 0u, 0u);
+                    fence_proxy_async_smem();
+                    next_tile(pf_l, pf_nt);
+                    pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->tempty[bsel]);
+                    if (lane == 0) mbar_arrive(&bars->tempty);
+                    sub(p_drain);
+                    // ---- the tile: first, without branches, every chunk's minimum, the
+                    //      tile's new best and window, and each chunk's count of other keys
+                    //      near the window; then the list insertions (one vote per tile) and,
+                    //      for the chunks that need them, the runner-up and further keys.
+                    //      Keys outside the window of a later (lower) best can never be
+                    //      candidates, so judging the whole tile against its final best is
+                    //      as rigorous as going chunk by chunk.
+                    const float inf = __int_as_float(0x7f800000);
+                    float kk[4][32];
+                    float c1k[4], g1[4];
 #pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2) {
-                        const int k0 = nt * BN + half * 64 + c2 * 32;
-                        const float4* cn4 = reinterpret_cast<const float4*>(cn + k0);
-                        float kk[32];
+                    for (int c2 = 0; c2 < 4; ++c2) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 c = cn4[q4];
-                            kk[4 * q4 + 0] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 0]), c.x), 4 * q4 + 0);
-                            kk[4 * q4 + 1] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 1]), c.y), 4 * q4 + 1);
-                            kk[4 * q4 + 2] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 2]), c.z), 4 * q4 + 2);
-                            kk[4 * q4 + 3] = local_key(fmaf(-2.f, __uint_as_float(v[c2][4 * q4 + 3]), c.w), 4 * q4 + 3);
-                        }
-                        const float c1k = min_of_32(kk);
-                        const float g1 = globalize(c1k, k0);
-                        // the key that loses the best slot (or the chunk minimum, if it
-                        // does not take it) joins the list when it is inside the window
-                        const float dem = fmaxf(cs.best, g1);
-                        cs.best = fminf(cs.best, g1);
-                        const float thr = cs.best + key_slack(cs.best) + twoE;
-                        const float inf = __int_as_float(0x7f800000);
-                        const bool dem_in = key_lower(dem) <= thr;
-                        if (kProf) ++n_chunk;
-                        if (__any_sync(0xffffffffu, dem_in)) {
-                            if (kProf) ++n_dem;
-                            cands_insert(cs, dem_in ? dem : inf);
-                        }
-                        // Any other key of the chunk inside the window? On the FMA pipe:
-                        // sum_j sat(kd (Td - key_j)), minus the minimum's own term. Td widens
-                        // thr by more than the key perturbations, and every key below Td adds
-                        // at least 2^-16, far above the rounding of the sum (<= 2^-18).
-                        const float Td = thr + 1.953125e-3f * (fabsf(thr) + twoE);
-                        const float kd = __fdividef(16.f, fabsf(Td) + twoE + 1e-30f);
-                        const float K = fmaf(kd, Td, 1.52587890625e-05f);
-                        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                        for (int j = 0; j < 32; ++j) kk[c2][j] = local_key(__uint_as_float(v[c2][j]), j);
+                        c1k[c2] = min_of_32(kk[c2]);
+                        g1[c2] = globalize(c1k[c2], nt * BN + half * 128 + c2 * 32);
+                    }
+                    const float old_best = cs.best;
+                    cs.best = fminf(old_best, fminf(fminf(g1[0], g1[1]), fminf(g1[2], g1[3])));
+                    const float thr = cs.best + key_slack(cs.best) + twoE;
+                    // Any other key of a chunk inside the window? On the FMA pipe:
+                    // sum_j sat(kd (Td - key_j)), minus the minimum's own term. Td widens thr
+                    // by more than the key perturbations, and every key below Td adds at
+                    // least 2^-16, far above the rounding of the sum (<= 2^-18).
+                    const float Td = thr + 1.953125e-3f * (fabsf(thr) + twoE);
+                    const float kd = __fdividef(16.f, fabsf(Td) + twoE + 1e-30f);
+                    const float K = fmaf(kd, Td, 1.52587890625e-05f);
+                    float other[4];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            a0 += fma_sat(-kd, kk[j + 0], K);
-                            a1 += fma_sat(-kd, kk[j + 1], K);
-                            a2 += fma_sat(-kd, kk[j + 2], K);
-                            a3 += fma_sat(-kd, kk[j + 3], K);
-                        }
-                        const float other = ((a0 + a1) + (a2 + a3)) - fma_sat(-kd, c1k, K);
-                        const bool second_cand = other > 9.5367431640625e-07f;  // 2^-20
+                    for (int c2 = 0; c2 < 4; ++c2) {
+                        float a[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a[i] = fma_sat(-kd, kk[c2][i], K);
+#pragma unroll
+                        for (int j = 8; j < 32; j += 8)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) a[i] += fma_sat(-kd, kk[c2][j + i], K);
+                        other[c2] = (((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]))) -
+                                    fma_sat(-kd, c1k[c2], K);
+                    }
+                    // the old best and the chunk minima, except the new best, join the list
+                    // when they are inside the window
+                    float ins[5];
+                    ins[0] = (old_best != cs.best && key_lower(old_best) <= thr) ? old_best : inf;
+#pragma unroll
+                    for (int c2 = 0; c2 < 4; ++c2)
+                        ins[1 + c2] = (g1[c2] != cs.best && key_lower(g1[c2]) <= thr) ? g1[c2] : inf;
+                    const bool any_in = fminf(fminf(ins[0], ins[1]), fminf(fminf(ins[2], ins[3]), ins[4])) < inf;
+                    if (kProf) n_chunk += 4;
+                    if (__any_sync(0xffffffffu, any_in)) {
+                        if (kProf) ++n_dem;
+#pragma unroll
+                        for (int i = 0; i < 5; ++i) cands_insert(cs, ins[i]);
+                    }
+#pragma unroll
+                    for (int c2 = 0; c2 < 4; ++c2) {
+                        const int k0 = nt * BN + half * 128 + c2 * 32;
+                        const bool second_cand = other[c2] > 9.5367431640625e-07f;  // 2^-20
                         if (__any_sync(0xffffffffu, second_cand)) {
                             if (kProf) ++n_sec;
                             // some lane has another key near the window: its runner-up goes
                             // in, and a third key is looked for only if the sum says so
                             float c1b, c2k;
-                            top2_of_32(kk, c1b, c2k);
+                            top2_of_32(kk[c2], c1b, c2k);
                             const float g2 = globalize(c2k, k0);
                             const bool second_in = second_cand && key_lower(g2) <= thr;
                             cands_insert(cs, second_in ? g2 : inf);
                             const bool more = second_cand &&
-                                              (other - fma_sat(-kd, c2k, K)) > 9.5367431640625e-07f;
+                                              (other[c2] - fma_sat(-kd, c2k, K)) > 9.5367431640625e-07f;
                             if (__any_sync(0xffffffffu, more)) {
                                 if (kProf) ++n_more;
                                 // further keys in ascending order (the keys are distinct: they
@@ -650,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int t = 0; t < TOPK - 2 && __any_sync(0xffffffffu, go); ++t) {
                                     float nk[32];
 #pragma unroll
-                                    for (int j = 0; j < 32; ++j) nk[j] = kk[j] > last ? kk[j] : inf;
+                                    for (int j = 0; j < 32; ++j) nk[j] = kk[c2][j] > last ? kk[c2][j] : inf;
                                     const float mn = min_of_32(nk);
                                     const float gn = globalize(mn, k0);
                                     const bool in = go && mn < inf && key_lower(gn) <= thr;
@@ -667,6 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 mark(p_scan);
+                t_sub = pclock<kProf>();
                 // ---- exchange both halves' lists; both merge them the same way
                 {
                     float* mine = xkeys + (half * BM + row) * 10;
@@ -677,7 +758,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ok = esync();
                 if (!ok) break;
-                if (l + 1 < n_q) stage_cn(l + 1);  // every read of this level's copy is done
                 {
                     const float* k0 = xkeys + row * 10;
                     const float* k1 = xkeys + (BM + row) * 10;
@@ -701,40 +781,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int slot = atomicAdd(rescan_count, 1);
                         if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
                     }
+                    sub(p_xchg);
+                    // ||c||^2 of the window's candidates for the pick, fetched now so that
+                    // the loads overlap the re-score
+                    float cnp[TOPK];
+#pragma unroll
+                    for (int p = 0; p < TOPK; ++p)
+                        cnp[p] = (m > 1 && p < m) ? __ldg(cnorm + (size_t)l * kK + key_index(cs.ts[p])) : 0.f;
                     // ---- float32 re-score of the window: each half dots its own 128
-                    //      dimensions of r with every candidate, 64 at a time
+                    //      dimensions of r with every candidate. The window entries are a
+                    //      prefix of the sorted list (m of them). r is read from TMEM 32
+                    //      dimensions at a time (one wait), and those dimensions of four
+                    //      candidates are fetched together (one L2 round trip per group).
                     float dot[TOPK];
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) dot[p] = 0.f;
-                    if (__any_sync(0xffffffffu, m > 1)) {
+                    int mw = m > 1 ? m : 0;  // candidates to re-score, warp maximum
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mw = max(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+                    if (mw > 0) {
+                        // row offsets of the candidates (lanes without a p-th read the best's row)
+                        uint32_t crow[TOPK];
+#pragma unroll
+                        for (int p = 0; p < TOPK; ++p)
+                            crow[p] = (uint32_t)key_index(m > 1 && p < m ? cs.ts[p] : cs.ts[0]) * kD +
+                                      half * 128;
 #pragma unroll 1
-                        for (int b = 0; b < 2; ++b) {
-                            uint32_t v[2][32];
-                            tmem_ld32(trow + (half * 4 + 2 * b) * 32, v[0]);
-                            tmem_ld32(trow + (half * 4 + 2 * b + 1) * 32, v[1]);
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t v[32];
+                            tmem_ld32(trow + half * 128 + q * 32, v);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int p = 0; p < TOPK; ++p) {
-                                if (m > 1 && key_lower(cs.ts[p]) <= wthr) {
-                                    const float4* c4 = reinterpret_cast<const float4*>(
-                                        book + (size_t)key_index(cs.ts[p]) * kD + half * 128 + b * 64);
-                                    float4 c[16];
+                            for (int pb = 0; pb < TOPK; pb += 4) {
+                                if (pb < mw) {
+                                    // only lanes with a (pb + j)-th candidate load it: the
+                                    // rows are scattered, so each lane's loads are separate
+                                    // L2 transactions
+                                    float4 c[4][8];
 #pragma unroll
-                                    for (int q4 = 0; q4 < 16; ++q4) c[q4] = __ldg(c4 + q4);
-                                    float a0 = 0.f, a1 = 0.f;
+                                    for (int j = 0; j < 4; ++j) {
+                                        const bool act = pb + j < m && m > 1;
+                                        const float4* c4 = reinterpret_cast<const float4*>(
+                                            book + crow[pb + j] + q * 32);
 #pragma unroll
-                                    for (int q4 = 0; q4 < 16; ++q4) {
-                                        const uint32_t* vv = v[q4 >> 3] + 4 * (q4 & 7);
-                                        a0 = fmaf(__uint_as_float(vv[0]), c[q4].x, a0);
-                                        a1 = fmaf(__uint_as_float(vv[1]), c[q4].y, a1);
-                                        a0 = fmaf(__uint_as_float(vv[2]), c[q4].z, a0);
-                                        a1 = fmaf(__uint_as_float(vv[3]), c[q4].w, a1);
+                                        for (int q4 = 0; q4 < 8; ++q4)
+                                            c[j][q4] = act ? __ldg(c4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
                                     }
-                                    dot[p] += a0 + a1;
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                                        for (int q4 = 0; q4 < 8; ++q4) {
+                                            a0 = fmaf(__uint_as_float(v[4 * q4 + 0]), c[j][q4].x, a0);
+                                            a1 = fmaf(__uint_as_float(v[4 * q4 + 1]), c[j][q4].y, a1);
+                                            a0 = fmaf(__uint_as_float(v[4 * q4 + 2]), c[j][q4].z, a0);
+                                            a1 = fmaf(__uint_as_float(v[4 * q4 + 3]), c[j][q4].w, a1);
+                                        }
+                                        dot[pb + j] += a0 + a1;
+                                    }
                                 }
                             }
                         }
                     }
+                    sub(p_rescore);
                     float* xd = xdot + (half * BM + row) * TOPK;
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) xd[p] = dot[p];
@@ -748,9 +857,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         int bw = 0x7fffffff;
 #pragma unroll
                         for (int p = 0; p < TOPK; ++p) {
-                            if (key_lower(cs.ts[p]) <= wthr) {
+                            if (p < m) {
                                 const int k = key_index(cs.ts[p]);
-                                const float e = fmaf(-2.f, d0[p] + d1[p], __ldg(cnorm + (size_t)l * kK + k));
+                                const float e = fmaf(-2.f, d0[p] + d1[p], cnp[p]);
                                 if (e < bs || (e == bs && k < bw)) {
                                     bs = e;
                                     bw = k;
@@ -760,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (bw < kK) win = bw;
                     }
                     win_codes[l] = win;
+                    sub(p_select);
                     mark(p_pick);
                     // ---- residual update r -= c_win for the next level, split by halves
                     if (updates_after(l)) {
@@ -768,27 +878,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         nr2 = 0.f;
                         ner2 = 0.f;
+                        // the winner's half-row with all 32 loads in flight (one round trip);
+                        // r read from TMEM 64 dimensions at a time
                         const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD + half * 128);
-#pragma unroll 1
-                        for (int b = 0; b < 2; ++b) {
-                            uint32_t v[2][32];
-                            tmem_ld32(trow + (half * 4 + 2 * b) * 32, v[0]);
-                            tmem_ld32(trow + (half * 4 + 2 * b + 1) * 32, v[1]);
-                            float4 c[16];
+                        float4 c[32];
 #pragma unroll
-                            for (int q4 = 0; q4 < 16; ++q4) c[q4] = __ldg(c4 + b * 16 + q4);
+                        for (int q4 = 0; q4 < 32; ++q4) c[q4] = __ldg(c4 + q4);
+#pragma unroll
+                        for (int b2 = 0; b2 < 2; ++b2) {
+                            uint32_t v[2][32];
+                            tmem_ld32(trow + (half * 4 + 2 * b2) * 32, v[0]);
+                            tmem_ld32(trow + (half * 4 + 2 * b2 + 1) * 32, v[1]);
                             tmem_wait_ld();
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
+                                const int c4i = 2 * b2 + h2;
+                                const int ch = half * 4 + c4i;
 #pragma unroll
                                 for (int q4 = 0; q4 < 8; ++q4) {
-                                    const float4 cc = c[h2 * 8 + q4];
+                                    const float4 cc = c[c4i * 8 + q4];
                                     v[h2][4 * q4 + 0] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 0]) - cc.x);
                                     v[h2][4 * q4 + 1] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 1]) - cc.y);
                                     v[h2][4 * q4 + 2] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 2]) - cc.z);
                                     v[h2][4 * q4 + 3] = __float_as_uint(__uint_as_float(v[h2][4 * q4 + 3]) - cc.w);
                                 }
-                                const int ch = half * 4 + 2 * b + h2;
                                 tmem_st32(trow + ch * 32, v[h2]);
                                 write_a_chunk(ch, v[h2], nr2, ner2);
                             }
@@ -821,13 +934,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         mark(p_stage);
-        if (kProf && prof && warp == 2 && lane == 0) {
+        if (kProf && prof && warp == kCtrlWarps && lane == 0) {
             atomicAdd(prof + P_EPI_TFULL, (unsigned long long)p_tfull);
             atomicAdd(prof + P_EPI_SCAN, (unsigned long long)p_scan);
             atomicAdd(prof + P_EPI_PICK, (unsigned long long)p_pick);
             atomicAdd(prof + P_EPI_UPDATE, (unsigned long long)p_update);
             atomicAdd(prof + P_EPI_STAGE, (unsigned long long)p_stage);
             atomicAdd(prof + P_EPI_ESYNC, (unsigned long long)p_esync);
+            atomicAdd(prof + P_PICK_XCHG, (unsigned long long)p_xchg);
+            atomicAdd(prof + P_PICK_RESCORE, (unsigned long long)p_rescore);
+            atomicAdd(prof + P_PICK_SELECT, (unsigned long long)p_select);
+            atomicAdd(prof + P_SCAN_DRAIN, (unsigned long long)p_drain);
         }
         if (kProf && prof && lane == 0) {
             atomicAdd(prof + P_N_CHUNK, n_chunk);
@@ -850,11 +967,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t encode_tc_configure() {
-    const cudaError_t e = cudaFuncSetAttribute(
-        k_encode_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_encode_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SMEM_BYTES);
+    for (auto* k : {k_encode_tc<false>, k_encode_tc<true>}) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        // the register split needs the launch allocation it was sized for
+        cudaFuncAttributes a;
+        e = cudaFuncGetAttributes(&a, k);
+        if (e != cudaSuccess) return e;
+        if (a.numRegs < kLaunchRegs || a.maxThreadsPerBlock < kThreads)
+            return cudaErrorLaunchOutOfResources;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
@@ -864,7 +987,8 @@ cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t 
     const int64_t tiles = (n + BM - 1) / BM;
     const int grid = (int)(tiles < max_ctas ? tiles : max_ctas);
     auto* kernel = prof ? k_encode_tc<true> : k_encode_tc<false>;
-    kernel<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm, t.cbound,
+    kernel<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm,
+                                              reinterpret_cast<const uint2*>(t.cnorm3), t.cbound,
                                               z, dtype, n, n_q, variant, codes, y_out, t.err,
                                               t.rescan_count, t.rescan_list, t.stats, prof);
     return cudaGetLastError();

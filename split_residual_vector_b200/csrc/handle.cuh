@@ -40,6 +40,7 @@ struct Tables {
     __nv_bfloat16* Win_hi = nullptr;  // [D][Din] bf16(W_in)
     __nv_bfloat16* Win_lo = nullptr;  // [D][Din] bf16(W_in - Win_hi)
     float* cnorm = nullptr;           // [Q][K] ||c||^2 (float64 sum, rounded)
+    __nv_bfloat16* cnorm3 = nullptr;  // [Q][K][4] (h, m, l, 0): h + m + l = cnorm / 2 exactly
     float* cbound = nullptr;          // [Q][4]: max ||c||, max ||c||^2, max ||bf16(c) - c||, 0 (rounded up)
     float* P = nullptr;               // [Q][K][Din] W_out . c (float64 sum, rounded): decode rows
     // device state
@@ -50,7 +51,7 @@ struct Tables {
     float* wide_y = nullptr;          // [kWideMaxFrames][D] latency encoder: projection exchange
     unsigned* wide_bars = nullptr;                // [kWideMaxGroups][kWideBarStride] group barriers
     unsigned long long* wide_partial = nullptr;   // per-CTA minimum keys, wide_partial_bytes()
-    // TMA descriptors (bf16, 64 x 128 boxes, 128-byte swizzle)
+    // TMA descriptors (bf16, 64 x 256 boxes, 128-byte swizzle)
     CUtensorMap tm_C;             // Cbf as [Q*K rows][D cols]
     CUtensorMap tm_Whi;           // Win_hi as [D rows][Din cols]
     CUtensorMap tm_Wlo;           // Win_lo

@@ -45,6 +45,24 @@ __global__ void k_norms(const float* __restrict__ C, float* __restrict__ cnorm,
     }
 }
 
+// ||c||^2 / 2 as three bf16 parts whose sum is exact (a float32 has 24
+// significant bits, each part takes the next 8): the B operand of the encode
+// kernel's norm step, which adds ||c||^2 / 2 to every score in the tensor core.
+__global__ void k_norm_split(const float* __restrict__ cnorm, __nv_bfloat16* __restrict__ out,
+                             int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float x = cnorm[i] * 0.5f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+    out[4 * i + 0] = h;
+    out[4 * i + 1] = m;
+    out[4 * i + 2] = l;
+    out[4 * i + 3] = __float2bfloat16_rn(0.f);
+}
+
 // W_in -> (hi, lo) bf16 split and a float32 transpose [Din][D].
 __global__ void k_split_win(const float* __restrict__ W, __nv_bfloat16* __restrict__ hi,
                             __nv_bfloat16* __restrict__ lo, float* __restrict__ WT) {
@@ -106,6 +124,7 @@ cudaError_t prep_tables(Tables& t, const float* W_out, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(t.cbound, 0, sizeof(float) * 4 * kQ, s);
     if (e != cudaSuccess) return e;
     k_norms<<<(kQ * kK * 32 + 255) / 256, 256, 0, s>>>(t.C32, t.cnorm, t.cbound);
+    k_norm_split<<<(kQ * kK + 255) / 256, 256, 0, s>>>(t.cnorm, t.cnorm3, kQ * kK);
     k_split_win<<<(kD * kDin + 255) / 256, 256, 0, s>>>(t.Win32, t.Win_hi, t.Win_lo, t.WinT32);
     dim3 grid(kDin / 64, kQ * kK / 64);
     k_decode_table<<<grid, 256, 0, s>>>(t.C32, W_out, t.P);

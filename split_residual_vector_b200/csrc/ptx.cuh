@@ -185,6 +185,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// K-major operand of 16 K elements (32 B per row) in the canonical layout
+// without swizzle: core matrices of 8 rows x 16 B, each stored as 128
+// contiguous bytes; the two K halves of an 8-row group 128 B apart (leading
+// byte offset), 8-row groups 256 B apart (stride byte offset).
+__device__ __forceinline__ uint32_t k16_offset(int row, int khalf) {
+    return (uint32_t)((row >> 3) * 256 + khalf * 128 + (row & 7) * 16);
+}
+
+// Shared-memory matrix descriptor of such an operand (layout type 0: no swizzle).
+__device__ __forceinline__ uint64_t k16_desc(uint32_t smem_addr) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
 // Instruction descriptor for kind::f16: bf16 A and B (both K-major), fp32 D,
 // shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
@@ -208,6 +222,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
           "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
           "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
           "=r"(v[31])
+        : "r"(taddr));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns (lane i: row lane base + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
 }
 
