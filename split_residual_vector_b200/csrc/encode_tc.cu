@@ -144,6 +144,7 @@ struct Bars {
     uint64_t zfull[2], zempty[2];
     uint64_t yfull, afull, aempty, drain;
     uint64_t tfull, tempty;     // the TMEM score buffer
+    uint64_t nready;            // the norm step's B tile holds the next score tile's norms
     uint64_t ebar;          // epilogue-wide barrier (all epilogue threads arrive)
     uint32_t tmem_base;
     int abort;
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&bars->tfull, 1);
         mbar_init(&bars->tempty, kEpiWarps);
+        mbar_init(&bars->nready, kEpiWarps);
         mbar_init(&bars->yfull, 1);
         mbar_init(&bars->afull, kEpiWarps);
         mbar_init(&bars->aempty, 1);
@@ -397,10 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t d = tmem + TMEM_SCORE;
-                        // ||c||^2 / 2 into the accumulator (the epilogue wrote this tile's
-                        // norms before releasing the buffer), then A = -bf16(r)
-                        umma_bf16(d, k16_desc(smem_u32(smem + ONESA_OFF)),
-                                  k16_desc(smem_u32(smem + NORMB_OFF)), idesc, 0u);
+                        // A = -bf16(r) over the 256 dimensions, then ||c||^2 / 2 added by the
+                        // norm step once the epilogue has written this tile's norms
                         for (int kc = 0; kc < KCH && ok; ++kc) {
                             const int s = it % STAGES;
                             ok = twait(&bars->full[s], (it / STAGES) & 1, p_full);
@@ -410,10 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t a = abase + kc * A_CHUNK_BYTES;
 #pragma unroll
                             for (int k = 0; k < BK / 16; ++k)
-                                umma_bf16(d, sw128_desc(a + 32 * k), sw128_desc(b + 32 * k), idesc, 1u);
+                                umma_bf16(d, sw128_desc(a + 32 * k), sw128_desc(b + 32 * k), idesc,
+                                          (kc > 0 || k > 0) ? 1u : 0u);
                             umma_commit(&bars->empty[s]);
                             ++it;
                         }
+                        if (!ok) break;
+                        ok = twait(&bars->nready, tcnt & 1, p_tempty);
+                        if (!ok) break;
+                        tc_fence_after();
+                        umma_bf16(d, k16_desc(smem_u32(smem + ONESA_OFF)),
+                                  k16_desc(smem_u32(smem + NORMB_OFF)), idesc, 1u);
                         umma_commit(&bars->tfull);
                         ++tcnt;
                     }
@@ -455,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         int pf_l = 0, pf_nt = 0;
         next_tile(pf_l, pf_nt);  // the setup wrote tile (0, 0); this is the one after it
+        if (lane == 0) mbar_arrive(&bars->nready);  // tile (0, 0)'s norms are in place
         uint2 pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
         float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
         float* xdot = reinterpret_cast<float*>(smem + XDOT_OFF);
@@ -637,19 +645,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // this half's 128 columns of the tile, all in registers: the buffer is
                     // released before the scan so that the next tile's MMAs run meanwhile
                     uint32_t v[4][32];
+                    {
+                        uint32_t w[2][64];
+                        tmem_ld64(trow + TMEM_SCORE + half * 128, w[0]);
+                        tmem_ld64(trow + TMEM_SCORE + half * 128 + 64, w[1]);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int c2 = 0; c2 < 4; ++c2)
-                        tmem_ld32(trow + TMEM_SCORE + half * 128 + c2 * 32, v[c2]);
-                    tmem_wait_ld();
-                    // the norm step of this tile has completed: write the next tile's norms
-                    *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(etid, 0)) =
-                        make_uint4(pf_norm.x, pf_norm.y, 0u, 0u);
-                    fence_proxy_async_smem();
-                    next_tile(pf_l, pf_nt);
-                    pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
+                        for (int j = 0; j < 128; ++j) v[j >> 5][j & 31] = w[j >> 6][j & 63];
+                    }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->tempty);
+                    // this tile's norm step has completed (it precedes the tile's commit):
+                    // write the next tile's norms; the MMA waits for them only at that
+                    // tile's norm step, after its 16 score MMAs
+                    *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(etid, 0)) =
+                        make_uint4(pf_norm.x, pf_norm.y, 0u, 0u);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->nready);
+                    next_tile(pf_l, pf_nt);
+                    pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
                     sub(p_drain);
                     // ---- the tile: first, without branches, every chunk's minimum, the
                     //      tile's new best and window, and each chunk's count of other keys
