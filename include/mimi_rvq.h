@@ -129,7 +129,7 @@ int mimi_rvq_encode_ex(mimi_rvq_t h, const void *latents, int dtype, int64_t N, 
 
 /*
  * Diagnostic: mimi_rvq_encode (n_q = 8, variant 0, N <= 1 048 576) that also
- * adds, into cycles[0..19] (device, caller-zeroed, uint64), the SM clock
+ * adds, into cycles[0..23] (device, caller-zeroed, uint64), the SM clock
  * cycles each role of the tensor-core kernel spent, summed over CTAs:
  *   0 TMA producer waiting for a free stage      1 MMA waiting for operand tiles
  *   2 MMA waiting for a drained score buffer     3 MMA waiting for a level's A operand
@@ -143,8 +143,10 @@ int mimi_rvq_encode_ex(mimi_rvq_t h, const void *latents, int dtype, int64_t N, 
  * lane 14 had a runner-up near the window, 15 had three or more keys near it; then
  * cycles again, as parts of 7: 16 list
  * exchange (its barrier included) and merge, 17 float32 re-score, 18 dot exchange and
- * the pick; and as part of 6: 19 copying a score tile to registers, writing the next
- * tile's norms and releasing the buffer. Codes are the same as mimi_rvq_encode's.
+ * the pick; as part of 6: 19 copying a score tile to registers, writing the next
+ * tile's norms and releasing the buffer; as parts of 8: 20 waiting for the MMA to
+ * finish with the A operand, 21 gather, subtract and stores, 22 combining the
+ * halves' norms; 23 unused. Codes are the same as mimi_rvq_encode's.
  */
 int mimi_rvq_encode_profile(mimi_rvq_t h, const void *latents, int dtype, int64_t N,
                             int16_t *codes, uint64_t *cycles, struct CUstream_st *stream);

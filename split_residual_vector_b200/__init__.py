@@ -223,7 +223,8 @@ class Quantizer:
                      "mma_wait_level_operand", "mma_wait_latents", "epi_wait_score_tile",
                      "epi_scan", "epi_pick", "epi_update", "epi_stage", "epi_barrier",
                      "cta_total", "n_chunks", "n_displaced", "n_runner_up", "n_more",
-                     "pick_exchange_merge", "pick_rescore", "pick_select", "scan_drain")
+                     "pick_exchange_merge", "pick_rescore", "pick_select", "scan_drain",
+                     "update_wait_operand", "update_work", "update_sync", "unused")
     PROFILE_COUNTS = ("n_chunks", "n_displaced", "n_runner_up", "n_more")
 
     def encode_profile(self, latents, out=None, stream=None):

@@ -136,7 +136,11 @@ enum ProfSlot {
     P_PICK_RESCORE,     //   float32 re-score of the window,
     P_PICK_SELECT,      //   dot exchange (barrier included) and the pick
     P_SCAN_DRAIN,       // part of P_EPI_SCAN: score tile to registers, next norms, release
-    kProfSlots = 20
+    P_UPD_AWAIT,        // parts of P_EPI_UPDATE: waiting for the MMA to finish with the A operand,
+    P_UPD_WORK,         //   gather, subtract, TMEM and A-operand stores,
+    P_UPD_SYNC,         //   combining the halves' norms (barrier included)
+    P_UNUSED,
+    kProfSlots = 24
 };
 
 struct Bars {
@@ -472,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned long long done = 0;
         long long p_tfull = 0, p_scan = 0, p_pick = 0, p_update = 0, p_stage = 0, p_esync = 0;
         long long p_xchg = 0, p_rescore = 0, p_select = 0, p_drain = 0, t_sub = 0;
+        long long p_uawait = 0, p_uwork = 0, p_usync = 0;
         // attribute the cycles since t_sub to one of the finer counters
         auto sub = [&](long long& acc) {
             const long long t = pclock<kProf>();
@@ -837,11 +842,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                     for (int j = 0; j < 4; ++j) {
                                         const bool act = pb + j < m && m > 1;
-                                        const float4* c4 = reinterpret_cast<const float4*>(
-                                            book + crow[pb + j] + q * 32);
+                                        const float* cp = book + crow[pb + j] + q * 32;
 #pragma unroll
-                                        for (int q4 = 0; q4 < 8; ++q4)
-                                            c[j][q4] = act ? __ldg(c4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                                        for (int q8 = 0; q8 < 4; ++q8) {
+                                            if (act) {
+                                                ldg_v8(cp + 8 * q8, c[j][2 * q8], c[j][2 * q8 + 1]);
+                                            } else {
+                                                c[j][2 * q8] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                                c[j][2 * q8 + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                            }
+                                        }
                                     }
 #pragma unroll
                                     for (int j = 0; j < 4; ++j) {
@@ -889,17 +899,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mark(p_pick);
                     // ---- residual update r -= c_win for the next level, split by halves
                     if (updates_after(l)) {
+                        t_sub = pclock<kProf>();
                         ok = ewait(&bars->aempty, aecnt & 1);
                         ++aecnt;
                         if (!ok) break;
+                        sub(p_uawait);
                         nr2 = 0.f;
                         ner2 = 0.f;
                         // the winner's half-row with all 32 loads in flight (one round trip);
                         // r read from TMEM 64 dimensions at a time
-                        const float4* c4 = reinterpret_cast<const float4*>(book + (size_t)win * kD + half * 128);
+                        const float* cw = book + (size_t)win * kD + half * 128;
                         float4 c[32];
 #pragma unroll
-                        for (int q4 = 0; q4 < 32; ++q4) c[q4] = __ldg(c4 + q4);
+                        for (int q8 = 0; q8 < 16; ++q8) ldg_v8(cw + 8 * q8, c[2 * q8], c[2 * q8 + 1]);
 #pragma unroll
                         for (int b2 = 0; b2 < 2; ++b2) {
                             uint32_t v[2][32];
@@ -927,8 +939,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bars->afull);
+                        sub(p_uwork);
                         ok = combine_norms(nr2, ner2);
                         if (!ok) break;
+                        sub(p_usync);
                         mark(p_update);
                     }
                 }
@@ -961,6 +975,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicAdd(prof + P_PICK_RESCORE, (unsigned long long)p_rescore);
             atomicAdd(prof + P_PICK_SELECT, (unsigned long long)p_select);
             atomicAdd(prof + P_SCAN_DRAIN, (unsigned long long)p_drain);
+            atomicAdd(prof + P_UPD_AWAIT, (unsigned long long)p_uawait);
+            atomicAdd(prof + P_UPD_WORK, (unsigned long long)p_uwork);
+            atomicAdd(prof + P_UPD_SYNC, (unsigned long long)p_usync);
         }
         if (kProf && prof && lane == 0) {
             atomicAdd(prof + P_N_CHUNK, n_chunk);

@@ -265,6 +265,15 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 32 bytes (8 floats) from global memory in one load (read-only path); p must be
+// 32-byte aligned. Halves the load instructions of a per-thread row gather.
+__device__ __forceinline__ void ldg_v8(const float* p, float4& lo, float4& hi) {
+    asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(lo.x), "=f"(lo.y), "=f"(lo.z), "=f"(lo.w), "=f"(hi.x), "=f"(hi.y),
+                   "=f"(hi.z), "=f"(hi.w)
+                 : "l"(p));
+}
+
 // ------------------------------------------------------------------ misc
 
 // Three-input float minimum (one instruction on sm_100a).
