@@ -554,7 +554,7 @@ def run_streaming(args):
     import split_residual_vector_b200 as pkg
     device = torch.device("cuda", 0)
     out = {}
-    for B in (1, 16, 128, 1024):
+    for B in args.batches:
         model, frames = synth.streaming_step(B, calls=args.calls)
         q = pkg.Quantizer(torch.from_numpy(model.C).to(device),
                           torch.from_numpy(model.W_in).to(device),
@@ -830,6 +830,8 @@ def main():
     ap.add_argument("--workload", default="encode_decode_1m", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--calls", type=int, default=1000, help="streaming workload: calls per B")
+    ap.add_argument("--batches", type=lambda v: [int(x) for x in v.split(",")],
+                    default=[1, 16, 128, 1024], help="streaming workload: the B values")
     ap.add_argument("--frames", type=int, default=None,
                     help="shrink the workload (for profiler captures); default: full size")
     ap.add_argument("--self-profile", action="store_true",

@@ -78,7 +78,7 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 void free_tables(mimi::Tables& t) {
     void* ptrs[] = {t.C32, t.Win32, t.WinT32, t.Cbf, t.Win_hi, t.Win_lo, t.cnorm, t.cnorm3, t.cbound,
                     t.P, t.err, t.rescan_count, t.rescan_list, t.stats, t.wide_y,
-                    t.wide_bars, t.wide_partial};
+                    t.wide_bars, t.wide_partial, t.slice_lists};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     const int sms = t.num_sms;
@@ -92,13 +92,14 @@ cudaError_t dalloc(T** p, size_t count) {
 }
 
 // Re-encode the frames the tensor-core kernel queued (count on the device) with
-// the float32 wide encoder, 1024 frames at a time.
+// the float32 wide encoder, `batch` frames at a time: 1024 after a batch encode
+// (hundreds of frames: 16 groups of 64 share the GPU), 64 after a streaming step
+// (usually none or one frame: one group spread over every SM finishes it fastest).
 cudaError_t rescan(mimi_rvq_t h, const void* z, int dtype, int n_q, int variant, int16_t* codes,
-                   cudaStream_t s) {
-    const mimi::WidePlan p = mimi::plan_encode_wide(mimi::kWideMaxFrames, h->num_sms);
+                   cudaStream_t s, int batch = mimi::kWideMaxFrames) {
+    const mimi::WidePlan p = mimi::plan_encode_wide(batch, h->num_sms);
     if (!p.ok) return cudaErrorInvalidConfiguration;
-    return mimi::launch_encode_wide(h->t, p, z, dtype, mimi::kWideMaxFrames, n_q, variant, codes,
-                                    s, true);
+    return mimi::launch_encode_wide(h->t, p, z, dtype, batch, n_q, variant, codes, s, true);
 }
 
 int check_common(mimi_rvq_t h, const void* in, const void* out, int64_t n) {
@@ -167,6 +168,9 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (e == cudaSuccess)
         e = cudaMalloc(reinterpret_cast<void**>(&t.wide_partial),
                        mimi::wide_partial_bytes(h->num_sms));
+    if (e == cudaSuccess)
+        e = dalloc(&t.slice_lists, (size_t)mimi::kSliceMaxGroups * mimi::kSlices * 128 *
+                                       mimi::kSliceListFloats);
     cudaStream_t s = nullptr;
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
     if (e == cudaSuccess)
@@ -242,6 +246,18 @@ int mimi_rvq_encode_step_ex(mimi_rvq_t h, const void* frames, int dtype, int B, 
     if (!h || B < 0) return MIMI_RVQ_EINVAL;
     if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
     if (n_q < 1 || n_q > kQ || (variant != 0 && variant != 1)) return MIMI_RVQ_EINVAL;
+    if (B >= mimi::kSlicedMinFrames && mimi::sliced_fits(B, h->num_sms)) {
+        // codebook-sliced tensor-core encode, then the float32 re-encode of the frames
+        // it could not certify
+        const int c = check_common(h, frames, codes, B);
+        if (c <= 0) return c;
+        cudaError_t e = cudaMemsetAsync(h->t.rescan_count, 0, sizeof(int), stream);
+        if (e == cudaSuccess)
+            e = mimi::launch_encode_tc_sliced(h->t, frames, dtype, B, n_q, variant, codes, stream);
+        if (e == cudaSuccess)
+            e = rescan(h, frames, dtype, n_q, variant, codes, stream, mimi::kWideGroupFrames);
+        return from_cuda(e);
+    }
     const mimi::WidePlan p = mimi::plan_encode_wide(B, h->num_sms);
     if (!p.ok) return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, n_q, variant, codes, stream);
     const int c = check_common(h, frames, codes, B);

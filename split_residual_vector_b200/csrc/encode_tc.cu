@@ -234,7 +234,13 @@ __device__ __forceinline__ long long pclock() {
 }
 
 // One CTA per SM (its shared memory and TMEM take the whole SM).
-template <bool kProf>
+// kSliced: the codebook-sliced form for streaming steps. CTA b serves frame
+// tile b / kSlices and, at every level, only score tile b % kSlices; after the
+// two halves have merged their lists, half 0 publishes the CTA's per-row list to
+// slice_lists, the group's CTAs meet at a bounded group barrier, and every CTA
+// merges the kSlices lists in slice order, so all of them certify, re-score and
+// pick the same codeword and keep the same residual. Slice 0 writes the codes.
+template <bool kProf, bool kSliced = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_encode_tc(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_Whi,
                 const __grid_constant__ CUtensorMap tm_Wlo, const float* __restrict__ C32,
@@ -243,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const void* __restrict__ z, int dtype, int64_t n, int n_q, int variant,
                 int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
                 int* rescan_count, int* rescan_list, unsigned long long* stats,
-                unsigned long long* prof) {
+                unsigned long long* prof, float* __restrict__ slice_lists, unsigned* slice_bars) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1 KiB alignment (128-byte swizzle atoms) as an offset into the shared
     // array, so that the compiler keeps the shared address space (LDS / STS)
@@ -254,6 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t abase = smem_u32(smem + A_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_tiles = (n + BM - 1) / BM;
+    // frame tiles of this CTA: blockIdx.x, + gridDim.x, ... (sliced: exactly one)
+    const int64_t tile_first = kSliced ? blockIdx.x / kSlices : blockIdx.x;
+    const int64_t tile_step = kSliced ? n_tiles : gridDim.x;
+    // score tiles of every level: all of them (sliced: this CTA's slice)
+    const int slice = kSliced ? (int)(blockIdx.x % kSlices) : 0;
+    const int nt_begin = kSliced ? slice : 0, nt_end = kSliced ? slice + 1 : NT;
     const bool f32_in = (dtype == 0);
     // Level l rewrites the A operand (r -= c_win, then bf16(r)) for level l + 1
     // when the next level quantises a different vector: always for acoustic
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);  // bf16 1, 1, 1, 0, ...
             *reinterpret_cast<uint4*>(smem + ONESA_OFF + k16_offset(i, 1)) = make_uint4(0u, 0u, 0u, 0u);
         }
-        const uint2 nv = __ldg(cnorm3 + i);
+        const uint2 nv = __ldg(cnorm3 + nt_begin * BN + i);
         *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(i, 0)) = make_uint4(nv.x, nv.y, 0u, 0u);
         *reinterpret_cast<uint4*>(smem + NORMB_OFF + k16_offset(i, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -330,11 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++it;
                 return true;
             };
-            for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            for (int64_t tile = tile_first; tile < n_tiles && ok; tile += tile_step) {
                 for (int kc = 0; kc < PKCH && ok; ++kc)
                     ok = ok && load(&tm_Whi, kc * BK, 0) && load(&tm_Wlo, kc * BK, 0);
                 for (int l = 0; l < n_q && ok; ++l)
-                    for (int nt = 0; nt < NT && ok; ++nt)
+                    for (int nt = nt_begin; nt < nt_end && ok; ++nt)
                         for (int kc = 0; kc < KCH && ok; ++kc)
                             ok = load(&tm_C, kc * BK, l * kK + nt * BN);
             }
@@ -357,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc += pclock<kProf>() - t0;
                 return r;
             };
-            for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            for (int64_t tile = tile_first; tile < n_tiles && ok; tile += tile_step) {
                 // projection: y = z_hi W_hi + z_lo W_hi + z_hi W_lo into columns [0, 256)
                 for (int kc = 0; kc < PKCH && ok; ++kc) {
                     const int zb = kc & 1;
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         tc_fence_after();
                     }
-                    for (int nt = 0; nt < NT && ok; ++nt) {
+                    for (int nt = nt_begin; nt < nt_end && ok; ++nt) {
                         ok = twait(&bars->tempty, (tcnt & 1) ^ 1, p_tempty);
                         if (!ok) break;
                         tc_fence_after();
@@ -459,12 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // draining one, thread etid writes its codeword's norm parts for the next into the
         // norm step's B tile. Each value is loaded one tile ahead of its write.
         auto next_tile = [&](int& l, int& nt) {
-            if (++nt == NT) {
-                nt = 0;
+            if (++nt == nt_end) {
+                nt = nt_begin;
                 if (++l == n_q) l = 0;
             }
         };
-        int pf_l = 0, pf_nt = 0;
+        int pf_l = 0, pf_nt = nt_begin;
         next_tile(pf_l, pf_nt);  // the setup wrote tile (0, 0); this is the one after it
         if (lane == 0) mbar_arrive(&bars->nready);  // tile (0, 0)'s norms are in place
         uint2 pf_norm = __ldg(cnorm3 + (size_t)pf_l * kK + pf_nt * BN + etid);
@@ -528,6 +540,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++ephase;
             return __all_sync(0xffffffffu, r) != 0;
         };
+        // Barrier of the group's CTAs (sliced form), among the epilogue threads only:
+        // every thread's list writes are fenced, the epilogue meets, one thread adds
+        // this CTA's arrival and (if wait) spins, bounded, until the count reaches
+        // target, and the epilogue meets again.
+        unsigned episode = 0;
+        auto group_sync = [&](unsigned* bar, unsigned target, bool wait) {
+            __threadfence();
+            if (!esync()) return false;
+            if (etid == 0) {
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+                if (wait) {
+                    const long long t0 = clock64();
+                    while (true) {
+                        unsigned v;
+                        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+                        if (v >= target) break;
+                        if (clock64() - t0 > kWaitBudgetCycles) {
+                            atomicOr(err, MIMI_DEV_ERR_TIMEOUT);
+                            *abort = 1;
+                            break;
+                        }
+                    }
+                    __threadfence();
+                }
+            }
+            if (!wait) return true;
+            return esync() && !*abort;
+        };
         // Both halves publish their partial norms; both read back the same sum.
         auto combine_norms = [&](float& nr2, float& ner2) {
             xnorm[(half * BM + row) * 2 + 0] = nr2;
@@ -538,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
 
-        for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tile_iter) {
+        for (int64_t tile = tile_first; tile < n_tiles && ok; tile += tile_step, ++tile_iter) {
             const int64_t frame = tile * BM + row;
             const bool valid = frame < n;
             // the A region is z staging now: wait for the previous tile's last MMAs
@@ -639,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Cands cs;
                 cands_reset(cs);
                 // ---- scan this half of the 8 score tiles of the codebook
-                for (int nt = 0; nt < NT; ++nt) {
+                for (int nt = nt_begin; nt < nt_end; ++nt) {
                     mark(p_scan);
                     ok = ewait(&bars->tfull, tcnt & 1);
                     mark(p_tfull);
@@ -791,13 +831,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cs.best = fminf(cs.best, best1);
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) cands_insert(cs, k1[p]);
+                    if constexpr (kSliced) {
+                        // publish this CTA's list of the row, meet the group's other slices,
+                        // then merge every slice's list (in slice order, so all slices get
+                        // the same list); after the last level only slice 0 goes on
+                        float* lists = slice_lists + (size_t)tile * kSlices * BM * kSliceListFloats;
+                        if (half == 0) {
+                            float* mine = lists + ((size_t)slice * BM + row) * kSliceListFloats;
+#pragma unroll
+                            for (int p = 0; p < TOPK; ++p) __stcg(mine + p, cs.ts[p]);
+                            __stcg(mine + 8, cs.best);
+                            __stcg(mine + 9, cs.evicted);
+                        }
+                        const bool last = l == n_q - 1;
+                        ++episode;
+                        ok = group_sync(slice_bars + tile * kWideBarStride, kSlices * episode,
+                                        !(last && slice != 0));
+                        if (!ok) break;
+                        if (last && slice != 0) break;
+                        // all slices' lists in one round trip, then merged in slice order
+                        float e[kSlices][kSliceListFloats];
+#pragma unroll
+                        for (int t = 0; t < kSlices; ++t) {
+                            const float* o = lists + ((size_t)t * BM + row) * kSliceListFloats;
+#pragma unroll
+                            for (int p = 0; p < kSliceListFloats; ++p) e[t][p] = __ldcg(o + p);
+                        }
+                        cands_reset(cs);
+#pragma unroll
+                        for (int t = 0; t < kSlices; ++t) {
+                            cs.evicted = fminf(cs.evicted, e[t][9]);
+                            cands_insert(cs, fmaxf(cs.best, e[t][8]));
+                            cs.best = fminf(cs.best, e[t][8]);
+#pragma unroll
+                            for (int p = 0; p < TOPK; ++p) cands_insert(cs, e[t][p]);
+                        }
+                        if (last && slice == 0 && etid == 0) atomicExch(slice_bars + tile * kWideBarStride, 0u);
+                    }
                     cands_insert(cs, cs.best);  // the best heads the candidate list
                     const float wthr = cs.best + key_slack(cs.best) + twoE;
                     int m = 0;
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) m += (key_lower(cs.ts[p]) <= wthr) ? 1 : 0;
                     const bool certified = key_lower(cs.evicted) > wthr;
-                    if (half == 0 && valid && !certified && !flagged) {
+                    if (half == 0 && valid && !certified && !flagged && (!kSliced || slice == 0)) {
                         flagged = true;
                         const int slot = atomicAdd(rescan_count, 1);
                         if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
@@ -949,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             tc_fence_before();
-            if (half == 0 && valid) {
+            if (half == 0 && valid && (!kSliced || slice == 0)) {
                 if (n_q == kQ) {
                     uint4 pk;
                     pk.x = (uint32_t)(uint16_t)win_codes[0] | ((uint32_t)(uint16_t)win_codes[1] << 16);
@@ -1000,7 +1077,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t encode_tc_configure() {
-    for (auto* k : {k_encode_tc<false>, k_encode_tc<true>}) {
+    for (auto* k : {k_encode_tc<false>, k_encode_tc<true>, k_encode_tc<false, true>}) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         // the register split needs the launch allocation it was sized for
@@ -1023,8 +1100,40 @@ cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t 
     kernel<<<grid, kThreads, SMEM_BYTES, s>>>(t.tm_C, t.tm_Whi, t.tm_Wlo, t.C32, t.cnorm,
                                               reinterpret_cast<const uint2*>(t.cnorm3), t.cbound,
                                               z, dtype, n, n_q, variant, codes, y_out, t.err,
-                                              t.rescan_count, t.rescan_list, t.stats, prof);
+                                              t.rescan_count, t.rescan_list, t.stats, prof,
+                                              nullptr, nullptr);
     return cudaGetLastError();
+}
+
+bool sliced_fits(int B, int num_sms) {
+    if (B <= 0 || B > BM * kSliceMaxGroups) return false;
+    return ((B + BM - 1) / BM) * kSlices <= num_sms;
+}
+
+cudaError_t launch_encode_tc_sliced(const Tables& t, const void* z, int dtype, int B, int n_q,
+                                    int variant, int16_t* codes, cudaStream_t s) {
+    if (!sliced_fits(B, t.num_sms)) return cudaErrorInvalidValue;
+    const int groups = (B + BM - 1) / BM;
+    CUtensorMap tm_C = t.tm_C, tm_Whi = t.tm_Whi, tm_Wlo = t.tm_Wlo;
+    const float* C32 = t.C32;
+    const float* cnorm = t.cnorm;
+    const uint2* cnorm3 = reinterpret_cast<const uint2*>(t.cnorm3);
+    const float* cbound = t.cbound;
+    int64_t n = B;
+    float* y_out = nullptr;
+    int* err = t.err;
+    int* rescan_count = t.rescan_count;
+    int* rescan_list = t.rescan_list;
+    unsigned long long* stats = t.stats;
+    unsigned long long* prof = nullptr;
+    float* lists = t.slice_lists;
+    unsigned* bars = t.wide_bars + kSliceBarBase * kWideBarStride;
+    void* args[] = {&tm_C, &tm_Whi, &tm_Wlo, &C32, &cnorm, &cnorm3, &cbound, &z, &dtype, &n,
+                    &n_q, &variant, &codes, &y_out, &err, &rescan_count, &rescan_list, &stats,
+                    &prof, &lists, &bars};
+    // every CTA of a group waits for the others: all must be resident at once
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_encode_tc<false, true>),
+                                       dim3(groups * kSlices), dim3(kThreads), args, SMEM_BYTES, s);
 }
 
 }  // namespace mimi

@@ -29,6 +29,19 @@ constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
 constexpr int kWideMaxGroups = 64;    // group barriers (the last one is the wait self-test's)
 constexpr int kWideBarStride = 32;    // words per group barrier (count, generation; own 128 B line)
 
+// Codebook-sliced form of the tensor-core encoder (streaming steps): each group
+// of up to 128 frames gets kSlices CTAs, one per 256-codeword score tile of a
+// level; the CTAs of a group exchange their candidate lists through global
+// memory behind a group barrier (group barriers kSliceBarBase .. + groups - 1 of
+// wide_bars, which the latency encoder and the wait self-test do not use).
+constexpr int kSlices = 8;
+constexpr int kSliceMaxGroups = 18;   // 18 x 8 CTAs fit on 148 SMs, one CTA each
+constexpr int kSliceBarBase = 32;
+constexpr int kSliceListFloats = 10;  // per row: 8 candidate keys, best, evicted
+// Streaming steps of at least this many frames take the sliced tensor-core
+// encoder (when its CTAs fit the device); smaller ones the float32 latency encoder.
+constexpr int kSlicedMinFrames = 512;
+
 struct Tables {
     int num_sms = 148;            // SMs of the handle's device (grid sizes)
     // float32 originals
@@ -51,6 +64,7 @@ struct Tables {
     float* wide_y = nullptr;          // [kWideMaxFrames][D] latency encoder: projection exchange
     unsigned* wide_bars = nullptr;                // [kWideMaxGroups][kWideBarStride] group barriers
     unsigned long long* wide_partial = nullptr;   // per-CTA minimum keys, wide_partial_bytes()
+    float* slice_lists = nullptr;   // [kSliceMaxGroups][kSlices][128][kSliceListFloats] sliced encoder
     // TMA descriptors (bf16, 64 x 256 boxes, 128-byte swizzle)
     CUtensorMap tm_C;             // Cbf as [Q*K rows][D cols]
     CUtensorMap tm_Whi;           // Win_hi as [D rows][Din cols]
@@ -67,6 +81,12 @@ cudaError_t encode_tc_configure();  // once per device, before the first launch
 cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                              int variant, int16_t* codes, float* y_out, cudaStream_t s,
                              int max_ctas, unsigned long long* prof = nullptr);
+// Codebook-sliced tensor-core encode of B frames (one cooperative launch of
+// ceil(B / 128) * kSlices CTAs); false from sliced_fits if B is outside
+// (0, 128 * kSliceMaxGroups] or the CTAs do not fit on the device at once.
+bool sliced_fits(int B, int num_sms);
+cudaError_t launch_encode_tc_sliced(const Tables& t, const void* z, int dtype, int B, int n_q,
+                                    int variant, int16_t* codes, cudaStream_t s);
 // encode_scan.cu
 cudaError_t launch_encode_scan(const Tables& t, const void* z, int dtype, int64_t n, int n_q,
                                int variant, int16_t* codes, cudaStream_t s);

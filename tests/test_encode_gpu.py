@@ -163,15 +163,16 @@ def test_streaming_step(batch):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_streaming_step_equals_full_scan(dtype):
-    """Small steps run the latency encoder, whose scores are the float32 full scan's (same
-    sums in the same order): every code equals encode_scan's, near ties included. Sizes span
-    one to 16 frame groups, ragged group tails and every thread-tile shape."""
+def test_small_streaming_steps_equal_the_full_scan(dtype):
+    """Steps under 512 frames run the latency encoder, whose scores are the float32 full
+    scan's (same sums in the same order): every code equals encode_scan's, near ties
+    included. Sizes span one to eight frame groups, ragged group tails and every thread-tile
+    shape."""
     model, frames = synth.streaming_step(1024, calls=1)
     q = quantizer(model)
     z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
     zd = to_device(np.ascontiguousarray(z))
-    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 896, 1000, 1024)
+    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 511)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         scan = q.encode_scan(zd[:b]).cpu().numpy()
@@ -181,20 +182,49 @@ def test_streaming_step_equals_full_scan(dtype):
     assert q.get_error() == 0
 
 
-def test_streaming_step_fewer_codebooks_and_variant():
-    model, frames = synth.streaming_step(300, calls=1)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sliced_streaming_steps_match_the_oracle(dtype):
+    """Steps of 512 frames and more run the codebook-sliced tensor-core encoder (8 CTAs per
+    128-frame group, candidate lists exchanged through global memory): codes equal the
+    oracle's outside near-ties and the batch tensor-core encoder's on every other frame,
+    for full and ragged groups, up to the 18 groups that fit the device at once."""
+    model, frames = synth.streaming_step(2304, calls=1)
     q = quantizer(model)
-    zd = to_device(np.ascontiguousarray(frames[0]))
-    for n_q, variant in ((1, 0), (5, 0), (8, 1), (3, 1)):
-        step = q.encode_step(zd, n_q=n_q, variant=variant).cpu().numpy()
-        scan = q.encode_scan(zd, n_q=n_q, variant=variant).cpu().numpy()
-        assert step.shape == (300, n_q) and np.array_equal(step, scan), (n_q, variant)
+    z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
+    zd = to_device(np.ascontiguousarray(z))
+    ref, db, ds = oracle.encode(z, model.W_in, model.C)
+    near = oracle.near_tie(db, ds)
+    enc0, _ = q.stats()
+    sizes = (512, 513, 700, 896, 1000, 1024, 2304)
+    for b in sizes:
+        step = q.encode_step(zd[:b]).cpu().numpy()
+        assert_codes_match(step, ref[:b], db[:b], ds[:b], f"sliced step B={b}")
+        batch = q.encode(zd[:b]).cpu().numpy()
+        differ = np.any(step != batch, axis=1)
+        assert not np.any(differ & ~near[:b]), f"B={b}: sliced and batch encoders differ off a near-tie"
+    enc, _ = q.stats()
+    assert enc - enc0 == 2 * sum(sizes)   # every step and every batch encode counted once
     assert q.get_error() == 0
 
 
-@pytest.mark.parametrize("batch", [1025, 5000])
-def test_streaming_step_large_batch_uses_the_batch_encoder(batch):
-    """Above the latency encoder's batch limit (1024) a step is a batch encode."""
+def test_streaming_step_fewer_codebooks_and_variant():
+    model, frames = synth.streaming_step(600, calls=1)
+    q = quantizer(model)
+    zd = to_device(np.ascontiguousarray(frames[0]))
+    for b in (100, 600):   # latency encoder, sliced tensor-core encoder
+        for n_q, variant in ((1, 0), (5, 0), (8, 1), (3, 1)):
+            step = q.encode_step(zd[:b], n_q=n_q, variant=variant).cpu().numpy()
+            assert step.shape == (b, n_q)
+            ref, db, ds = oracle.encode(frames[0][:b], model.W_in, model.C, n_q=n_q,
+                                        variant=variant)
+            assert_codes_match(step, ref, db, ds, f"step B={b} n_q={n_q} variant={variant}")
+    assert q.get_error() == 0
+
+
+@pytest.mark.parametrize("batch", [1025, 2305, 5000])
+def test_streaming_step_large_batch(batch):
+    """Up to 2304 frames (18 groups of 8 CTAs on 148 SMs) a step is sliced; above, a batch
+    encode."""
     model, frames = synth.streaming_step(batch, calls=1)
     q = quantizer(model)
     codes = q.encode_step(to_device(np.ascontiguousarray(frames[0]))).cpu().numpy()
@@ -204,10 +234,11 @@ def test_streaming_step_large_batch_uses_the_batch_encoder(batch):
     assert q.get_error() == 0
 
 
-@pytest.mark.parametrize("batch", [1, 128])
+@pytest.mark.parametrize("batch", [1, 128, 1024])
 def test_streaming_step_in_a_cuda_graph(batch):
-    """The latency encoder's group barriers return to their starting state after every
-    launch, so a captured step replays correctly on new inputs."""
+    """The group barriers of both streaming encoders return to their starting state after
+    every launch, so a captured step replays correctly on new inputs (the same codes as an
+    uncaptured step)."""
     model, frames = synth.streaming_step(batch, calls=4)
     q = quantizer(model)
     static_in = to_device(np.ascontiguousarray(frames[0]))
@@ -226,8 +257,10 @@ def test_streaming_step_in_a_cuda_graph(batch):
         g.replay()
         torch.cuda.synchronize()
         got = static_out.cpu().numpy()
-        want = q.encode_scan(static_in).cpu().numpy()
+        want = q.encode_step(static_in).cpu().numpy()
         assert np.array_equal(got, want), f"replay {call}"
+        ref, db, ds = oracle.encode(frames[call], model.W_in, model.C)
+        assert_codes_match(got, ref, db, ds, f"replay {call}")
     assert q.get_error() == 0
 
 
