@@ -78,10 +78,10 @@ MOSHI_DELAYS = [0, 1, 1, 1, 1, 1, 1, 1]   # acoustic delay 1 (the final model's)
 # DRAM bytes (read + write) per unit from one ncu capture of the current kernel, with the
 # summary that records it; the bench scales it by the units of a launch. None: not captured.
 NCU_TRAFFIC_PER_UNIT = {
-    "k_embed_sum": (48_951, "profiles/k_embed_sum_moshi_input.md"),        # per step
-    "k_encode_tc/f32": (2_478, "profiles/k_encode_tc_offline_batch.md"),   # per fp32 frame
-    "k_encode_tc/bf16": (1_161, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
-    "k_decode": (1_990, "profiles/k_decode_decode_heavy.md"),              # per frame
+    "k_embed_sum": (48_927, "profiles/k_embed_sum_moshi_input.md"),        # per step
+    "k_encode_tc/f32": (2_488, "profiles/k_encode_tc_offline_batch_fp32.md"),  # per fp32 frame
+    "k_encode_tc/bf16": (1_163, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
+    "k_decode": (1_987, "profiles/k_decode_decode_heavy.md"),              # per frame
 }
 
 
@@ -484,6 +484,7 @@ def run_ours(args, rank, world, local_rank):
     lat_bytes = 2048 if lat_dtype == "f32" else 1024
     if do_enc:
         tf = enc_flop(n_q) * n / (enc_avg / 1e3) / 1e12
+        f_enc, f_re = q_enc.stats()    # since create: warm-up, timed and e2e calls
         # the captured DRAM traffic is for the full 8-codebook, variant-0 encode
         tr = (NCU_TRAFFIC_PER_UNIT.get("k_encode_tc/" + lat_dtype)
               if (n_q, variant) == (8, 0) else None)
@@ -495,6 +496,7 @@ def run_ours(args, rank, world, local_rank):
             "traffic": tr[0] * n if tr and tr[0] else None,
             "traffic_source": tr[1] if tr and tr[0] else None,
             "ms": enc_avg, "frames": n, "latent_dtype": lat_dtype,
+            "reencoded_frames_per_call": f_re / f_enc * n if f_enc else None,
             "algorithmic": (f"{enc_flop(n_q)} FLOP/frame x {n} frames; "
                             f"HBM {lat_bytes + 2 * n_q} B/frame"),
             "hbm_gbs": (lat_bytes + 2 * n_q) * n / (enc_avg / 1e3) / 1e9})
