@@ -78,7 +78,7 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 void free_tables(mimi::Tables& t) {
     void* ptrs[] = {t.C32, t.Win32, t.WinT32, t.Cbf, t.Win_hi, t.Win_lo, t.cnorm, t.cnorm3, t.cbound,
                     t.P, t.err, t.rescan_count, t.rescan_list, t.stats, t.wide_y,
-                    t.wide_bars, t.wide_partial, t.slice_lists};
+                    t.wide_bars, t.wide_partial, t.slice_lists, t.slice_exact};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     const int sms = t.num_sms;
@@ -91,12 +91,11 @@ cudaError_t dalloc(T** p, size_t count) {
     return cudaMalloc(reinterpret_cast<void**>(p), sizeof(T) * count);
 }
 
-// Re-encode the frames the tensor-core kernel queued (count on the device) with
-// the float32 wide encoder, `batch` frames at a time: 1024 after a batch encode
-// (hundreds of frames: 16 groups of 64 share the GPU), 64 after a streaming step
-// (usually none or one frame: one group spread over every SM finishes it fastest).
+// Re-encode the frames the batch tensor-core kernel queued (count on the device)
+// with the float32 wide encoder, 1024 at a time (16 groups of 64 share the GPU).
 cudaError_t rescan(mimi_rvq_t h, const void* z, int dtype, int n_q, int variant, int16_t* codes,
-                   cudaStream_t s, int batch = mimi::kWideMaxFrames) {
+                   cudaStream_t s) {
+    const int batch = mimi::kWideMaxFrames;
     const mimi::WidePlan p = mimi::plan_encode_wide(batch, h->num_sms);
     if (!p.ok) return cudaErrorInvalidConfiguration;
     return mimi::launch_encode_wide(h->t, p, z, dtype, batch, n_q, variant, codes, s, true);
@@ -169,8 +168,10 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
         e = cudaMalloc(reinterpret_cast<void**>(&t.wide_partial),
                        mimi::wide_partial_bytes(h->num_sms));
     if (e == cudaSuccess)
-        e = dalloc(&t.slice_lists, (size_t)mimi::kSliceMaxGroups * mimi::kSlices * 128 *
+        e = dalloc(&t.slice_lists, (size_t)2 * mimi::kSliceMaxGroups * mimi::kSlices * 128 *
                                        mimi::kSliceListFloats);
+    if (e == cudaSuccess)
+        e = dalloc(&t.slice_exact, (size_t)mimi::kSliceMaxGroups * 128 * mimi::kSlices);
     cudaStream_t s = nullptr;
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
     if (e == cudaSuccess)
@@ -247,16 +248,12 @@ int mimi_rvq_encode_step_ex(mimi_rvq_t h, const void* frames, int dtype, int B, 
     if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
     if (n_q < 1 || n_q > kQ || (variant != 0 && variant != 1)) return MIMI_RVQ_EINVAL;
     if (B >= mimi::kSlicedMinFrames && mimi::sliced_fits(B, h->num_sms)) {
-        // codebook-sliced tensor-core encode, then the float32 re-encode of the frames
-        // it could not certify
+        // codebook-sliced tensor-core encode (rows it cannot certify take an exact
+        // float32 scan inside the kernel: one launch)
         const int c = check_common(h, frames, codes, B);
         if (c <= 0) return c;
-        cudaError_t e = cudaMemsetAsync(h->t.rescan_count, 0, sizeof(int), stream);
-        if (e == cudaSuccess)
-            e = mimi::launch_encode_tc_sliced(h->t, frames, dtype, B, n_q, variant, codes, stream);
-        if (e == cudaSuccess)
-            e = rescan(h, frames, dtype, n_q, variant, codes, stream, mimi::kWideGroupFrames);
-        return from_cuda(e);
+        return from_cuda(
+            mimi::launch_encode_tc_sliced(h->t, frames, dtype, B, n_q, variant, codes, stream));
     }
     const mimi::WidePlan p = mimi::plan_encode_wide(B, h->num_sms);
     if (!p.ok) return mimi_rvq_encode_ex(h, frames, dtype, (int64_t)B, n_q, variant, codes, stream);

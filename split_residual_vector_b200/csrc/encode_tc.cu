@@ -68,7 +68,10 @@ constexpr int XNORM_OFF = XDOT_OFF + 2 * BM * TOPK * 4; // [2][BM][2] partial no
 constexpr int NORMB_OFF = XNORM_OFF + 2 * BM * 2 * 4;  // [BN][16] bf16
 constexpr int ONESA_OFF = NORMB_OFF + BN * 32;         // [BM][16] bf16
 constexpr int BAR_OFF = ONESA_OFF + BM * 32;
-constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;        // barriers, slack for 1 KiB alignment
+// The rows of a level whose candidate set could not be certified: one bit per
+// row, a 32-bit word per TMEM lane quarter.
+constexpr int UMASK_OFF = BAR_OFF + 512;
+constexpr int SMEM_BYTES = UMASK_OFF + 64 + 1024;  // slack for 1 KiB alignment
 constexpr int kEpiWarps = 8;            // two per TMEM lane quarter: column halves
 constexpr int kCtrlWarps = 4;           // warpgroup 0: TMA (warp 0), MMA (warp 1), two idle
 constexpr int kThreads = 32 * (kCtrlWarps + kEpiWarps);   // 384: three warpgroups
@@ -249,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const void* __restrict__ z, int dtype, int64_t n, int n_q, int variant,
                 int16_t* __restrict__ codes, float* __restrict__ y_out, int* err,
                 int* rescan_count, int* rescan_list, unsigned long long* stats,
-                unsigned long long* prof, float* __restrict__ slice_lists, unsigned* slice_bars) {
+                unsigned long long* prof, float* __restrict__ slice_lists, unsigned* slice_bars,
+                float2* __restrict__ slice_exact) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1 KiB alignment (128-byte swizzle atoms) as an offset into the shared
     // array, so that the compiler keeps the shared address space (LDS / STS)
@@ -483,6 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* xkeys = reinterpret_cast<float*>(smem + XKEYS_OFF);
         float* xdot = reinterpret_cast<float*>(smem + XDOT_OFF);
         float* xnorm = reinterpret_cast<float*>(smem + XNORM_OFF);
+        volatile unsigned* s_umask = reinterpret_cast<volatile unsigned*>(smem + UMASK_OFF);
+        // the exact scan of an uncertified row: the row's r (256 floats) and each warp's
+        // best, in the list-exchange area (free from the re-score on; see below)
+        float* s_r = xkeys;
+        float* s_bs = xkeys + kD;
+        int* s_bk = reinterpret_cast<int*>(xkeys + kD + kEpiWarps);
         uint32_t zuse[2] = {0, 0}, aecnt = 0, tcnt = 0, tile_iter = 0;
         bool ok = true;
         unsigned long long done = 0;
@@ -835,7 +845,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // publish this CTA's list of the row, meet the group's other slices,
                         // then merge every slice's list (in slice order, so all slices get
                         // the same list); after the last level only slice 0 goes on
-                        float* lists = slice_lists + (size_t)tile * kSlices * BM * kSliceListFloats;
+                        // two buffers by level parity: a slice that has raced ahead to the next
+                        // level's publication never overwrites lists a slower slice still reads
+                        // (no group barrier need separate the two when no row needs the exact scan)
+                        float* lists = slice_lists +
+                                       ((size_t)(l & 1) * kSliceMaxGroups + tile) * kSlices * BM * kSliceListFloats;
                         if (half == 0) {
                             float* mine = lists + ((size_t)slice * BM + row) * kSliceListFloats;
 #pragma unroll
@@ -843,12 +857,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __stcg(mine + 8, cs.best);
                             __stcg(mine + 9, cs.evicted);
                         }
-                        const bool last = l == n_q - 1;
                         ++episode;
-                        ok = group_sync(slice_bars + tile * kWideBarStride, kSlices * episode,
-                                        !(last && slice != 0));
+                        ok = group_sync(slice_bars + tile * kWideBarStride, kSlices * episode, true);
                         if (!ok) break;
-                        if (last && slice != 0) break;
                         // all slices' lists in one round trip, then merged in slice order
                         float e[kSlices][kSliceListFloats];
 #pragma unroll
@@ -866,7 +877,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int p = 0; p < TOPK; ++p) cands_insert(cs, e[t][p]);
                         }
-                        if (last && slice == 0 && etid == 0) atomicExch(slice_bars + tile * kWideBarStride, 0u);
                     }
                     cands_insert(cs, cs.best);  // the best heads the candidate list
                     const float wthr = cs.best + key_slack(cs.best) + twoE;
@@ -874,10 +884,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int p = 0; p < TOPK; ++p) m += (key_lower(cs.ts[p]) <= wthr) ? 1 : 0;
                     const bool certified = key_lower(cs.evicted) > wthr;
-                    if (half == 0 && valid && !certified && !flagged && (!kSliced || slice == 0)) {
-                        flagged = true;
-                        const int slot = atomicAdd(rescan_count, 1);
-                        if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
+                    if constexpr (kSliced) {
+                        // uncertified rows are marked for the exact scan below (every word is
+                        // rewritten at every level); the statistic counts each such frame once
+                        if (half == 0) {
+                            const unsigned um = __ballot_sync(0xffffffffu, valid && !certified);
+                            if (lane == 0) s_umask[quarter] = um;
+                            if (valid && !certified && !flagged && slice == 0) atomicAdd(&stats[1], 1ull);
+                        }
+                        flagged = flagged || !certified;
+                    } else {
+                        // the frame is queued for the float32 re-encode after this kernel (an
+                        // exact scan here would read the whole float32 codebook per row)
+                        if (half == 0 && valid && !certified && !flagged) {
+                            flagged = true;
+                            const int slot = atomicAdd(rescan_count, 1);
+                            if (slot < (int)kRescanCapacity) rescan_list[slot] = (int)frame;
+                        }
                     }
                     sub(p_xchg);
                     // ||c||^2 of the window's candidates for the pick, fetched now so that
@@ -970,6 +993,138 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         if (bw < kK) win = bw;
+                    }
+                    // ---- sliced: rows whose candidate set could not be certified (more window
+                    //      keys than the list holds) take an exact float32 scan of the slice's
+                    //      256 codewords, row by row, instead of a re-encode after the kernel.
+                    //      The row's r goes through shared memory; each warp takes 32
+                    //      codewords (lane j: dimensions 8 j .. 8 j + 7 of a row, a coalesced
+                    //      1 KiB load, then a butterfly sum); the lowest score wins, ties to the
+                    //      lowest index, over the warps and then over the group's slices. Rows
+                    //      go in ascending order, the same in every slice of a group.
+                    unsigned um[4] = {0u, 0u, 0u, 0u};
+                    int nu = 0;
+                    if constexpr (kSliced) {
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            um[w] = s_umask[w];
+                            nu += __popc(um[w]);
+                        }
+                    }
+                    for (int i = 0; i < nu; ++i) {
+                        int u = 0;
+#pragma unroll
+                        for (int w = 3; w >= 0; --w)  // the lowest marked row left
+                            if (um[w]) u = w * 32 + __ffs(um[w]) - 1;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            if (w == (u >> 5)) um[w] &= um[w] - 1;
+                        if (quarter == (u >> 5)) {  // both warps of u's lane quarter (warp-uniform)
+#pragma unroll 1
+                            for (int c4 = 0; c4 < 4; ++c4) {
+                                uint32_t v[32];
+                                tmem_ld32(trow + (half * 4 + c4) * 32, v);
+                                tmem_wait_ld();
+                                if (lane == (u & 31)) {
+                                    float4* dst = reinterpret_cast<float4*>(s_r + (half * 4 + c4) * 32);
+#pragma unroll
+                                    for (int q4 = 0; q4 < 8; ++q4)
+                                        dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                                              __uint_as_float(v[4 * q4 + 2]),
+                                                              __uint_as_float(v[4 * q4 + 3]));
+                                }
+                            }
+                        }
+                        ok = esync();
+                        if (!ok) break;
+                        const int ew = etid >> 5;
+                        constexpr int kn = BN / kEpiWarps;   // codewords per warp
+                        const int kb = nt_begin * BN + ew * kn;
+                        const float4 ra = reinterpret_cast<const float4*>(s_r)[2 * lane];
+                        const float4 rb = reinterpret_cast<const float4*>(s_r)[2 * lane + 1];
+                        float bs = __int_as_float(0x7f800000);
+                        int bk = 0x7fffffff;
+                        // 16 codeword rows per step in flight (one at a time would be bound by
+                        // the latency of each load)
+                        constexpr int kRows = 16;
+#pragma unroll 1
+                        for (int j0 = 0; j0 < kn; j0 += kRows) {
+                            float4 ca[kRows], cb[kRows];
+                            float cn[kRows];
+#pragma unroll
+                            for (int t = 0; t < kRows; ++t) {
+                                ldg_v8(book + (size_t)(kb + j0 + t) * kD + 8 * lane, ca[t], cb[t]);
+                                cn[t] = __ldg(cnorm + (size_t)l * kK + kb + j0 + t);
+                            }
+#pragma unroll
+                            for (int t = 0; t < kRows; ++t) {
+                                float d = ra.x * ca[t].x;
+                                d = fmaf(ra.y, ca[t].y, d);
+                                d = fmaf(ra.z, ca[t].z, d);
+                                d = fmaf(ra.w, ca[t].w, d);
+                                d = fmaf(rb.x, cb[t].x, d);
+                                d = fmaf(rb.y, cb[t].y, d);
+                                d = fmaf(rb.z, cb[t].z, d);
+                                d = fmaf(rb.w, cb[t].w, d);
+#pragma unroll
+                                for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                                const float e = fmaf(-2.f, d, cn[t]);
+                                if (e < bs) {  // codewords ascending: a tie keeps the lower index
+                                    bs = e;
+                                    bk = kb + j0 + t;
+                                }
+                            }
+                        }
+                        if (lane == 0) {
+                            s_bs[ew] = bs;
+                            s_bk[ew] = bk;
+                        }
+                        ok = esync();
+                        if (!ok) break;
+                        float gb = __int_as_float(0x7f800000);
+                        int gk = 0x7fffffff;
+#pragma unroll
+                        for (int w = 0; w < kEpiWarps; ++w) {
+                            const float e = s_bs[w];
+                            const int k = s_bk[w];
+                            if (e < gb || (e == gb && k < gk)) {
+                                gb = e;
+                                gk = k;
+                            }
+                        }
+                        if constexpr (kSliced) {
+                            float2* ex = slice_exact + ((size_t)tile * BM + u) * kSlices;
+                            if (etid == 0) __stcg(ex + slice, make_float2(gb, __int_as_float(gk)));
+                            ++episode;
+                            ok = group_sync(slice_bars + tile * kWideBarStride, kSlices * episode, true);
+                            if (!ok) break;
+                            gb = __int_as_float(0x7f800000);
+                            gk = 0x7fffffff;
+#pragma unroll
+                            for (int t = 0; t < kSlices; ++t) {
+                                const float2 x = __ldcg(ex + t);
+                                const int k = __float_as_int(x.y);
+                                if (x.x < gb || (x.x == gb && k < gk)) {
+                                    gb = x.x;
+                                    gk = k;
+                                }
+                            }
+                        }
+                        if (row == u && gk < kK) win = gk;
+                        ok = esync();  // s_r and the warp bests are rewritten for the next row
+                        if (!ok) break;
+                    }
+                    if (!ok) break;
+                    if constexpr (kSliced) {
+                        // the group's last arrival: slice 0 waits for all of them, then resets
+                        // the counter for the next launch
+                        if (l == n_q - 1) {
+                            ++episode;
+                            ok = group_sync(slice_bars + tile * kWideBarStride, kSlices * episode,
+                                            slice == 0);
+                            if (!ok) break;
+                            if (slice == 0 && etid == 0) atomicExch(slice_bars + tile * kWideBarStride, 0u);
+                        }
                     }
                     win_codes[l] = win;
                     sub(p_select);
@@ -1101,7 +1256,7 @@ cudaError_t launch_encode_tc(const Tables& t, const void* z, int dtype, int64_t 
                                               reinterpret_cast<const uint2*>(t.cnorm3), t.cbound,
                                               z, dtype, n, n_q, variant, codes, y_out, t.err,
                                               t.rescan_count, t.rescan_list, t.stats, prof,
-                                              nullptr, nullptr);
+                                              nullptr, nullptr, nullptr);
     return cudaGetLastError();
 }
 
@@ -1128,9 +1283,10 @@ cudaError_t launch_encode_tc_sliced(const Tables& t, const void* z, int dtype, i
     unsigned long long* prof = nullptr;
     float* lists = t.slice_lists;
     unsigned* bars = t.wide_bars + kSliceBarBase * kWideBarStride;
+    float2* exact = t.slice_exact;
     void* args[] = {&tm_C, &tm_Whi, &tm_Wlo, &C32, &cnorm, &cnorm3, &cbound, &z, &dtype, &n,
                     &n_q, &variant, &codes, &y_out, &err, &rescan_count, &rescan_list, &stats,
-                    &prof, &lists, &bars};
+                    &prof, &lists, &bars, &exact};
     // every CTA of a group waits for the others: all must be resident at once
     return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_encode_tc<false, true>),
                                        dim3(groups * kSlices), dim3(kThreads), args, SMEM_BYTES, s);

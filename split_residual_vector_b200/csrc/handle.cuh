@@ -64,7 +64,8 @@ struct Tables {
     float* wide_y = nullptr;          // [kWideMaxFrames][D] latency encoder: projection exchange
     unsigned* wide_bars = nullptr;                // [kWideMaxGroups][kWideBarStride] group barriers
     unsigned long long* wide_partial = nullptr;   // per-CTA minimum keys, wide_partial_bytes()
-    float* slice_lists = nullptr;   // [kSliceMaxGroups][kSlices][128][kSliceListFloats] sliced encoder
+    float* slice_lists = nullptr;   // [2][kSliceMaxGroups][kSlices][128][kSliceListFloats] sliced encoder
+    float2* slice_exact = nullptr;  // [kSliceMaxGroups][128][kSlices] sliced encoder: exact-scan bests
     // TMA descriptors (bf16, 64 x 256 boxes, 128-byte swizzle)
     CUtensorMap tm_C;             // Cbf as [Q*K rows][D cols]
     CUtensorMap tm_Whi;           // Win_hi as [D rows][Din cols]

@@ -207,6 +207,30 @@ def test_sliced_streaming_steps_match_the_oracle(dtype):
     assert q.get_error() == 0
 
 
+def test_sliced_step_uncertified_rows_take_the_exact_scan():
+    """Every level-1 codeword has ~20 exact copies, so no row of a sliced streaming step can
+    certify its candidate window at level 1: each takes the in-kernel exact float32 scan of
+    every slice's codewords, merged over the group (ties between copies go to the lowest
+    index). 600 frames: four full groups and a ragged one. The codes match the oracle, and the
+    float32 full-scan kernel's off the oracle's near-ties; each frame is counted once."""
+    model = _small_model(seed=33)
+    model.C[1] = model.C[1][np.arange(2048) % 100]
+    q = quantizer(model)
+    rng = np.random.default_rng(36)
+    z = rng.standard_normal((600, 512)).astype(np.float32)
+    zd = to_device(z)
+    codes = q.encode_step(zd).cpu().numpy()
+    assert q.get_error() == 0
+    _, uncertified = q.stats()
+    assert uncertified == 600
+    ref, db, ds = oracle.encode(z, model.W_in, model.C)
+    assert_codes_match(codes, ref, db, ds, "sliced, all rows uncertified")
+    assert (codes[:, 1] < 100).all()  # the lowest of the tied copies
+    near = oracle.near_tie(db, ds)
+    scan = q.encode_scan(zd).cpu().numpy()
+    assert np.array_equal(codes[~near], scan[~near])
+
+
 def test_streaming_step_fewer_codebooks_and_variant():
     model, frames = synth.streaming_step(600, calls=1)
     q = quantizer(model)
