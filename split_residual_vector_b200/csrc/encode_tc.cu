@@ -556,9 +556,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // target, and the epilogue meets again.
         unsigned episode = 0;
         auto group_sync = [&](unsigned* bar, unsigned target, bool wait) {
-            __threadfence();
+            // the CTA meets first; then one thread fences (which orders every write the
+            // CTA barrier ordered before it) and arrives, as a grid-wide barrier does
             if (!esync()) return false;
             if (etid == 0) {
+                __threadfence();
                 asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
                 if (wait) {
                     const long long t0 = clock64();
