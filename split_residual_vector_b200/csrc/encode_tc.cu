@@ -193,12 +193,9 @@ __device__ __forceinline__ void cx(float& a, float& b) {
     b = fmaxf(a, b);
     a = lo;
 }
-__device__ __forceinline__ void cands_insert5(Cands& c, const float (&k)[5]) {
-    const float inf = __int_as_float(0x7f800000);
-    float s[8] = {k[0], k[1], k[2], k[3], k[4], inf, inf, inf};
-    cx(s[0], s[1]); cx(s[3], s[4]); cx(s[2], s[4]);
-    cx(s[2], s[3]); cx(s[0], s[3]); cx(s[0], s[2]);
-    cx(s[1], s[4]); cx(s[1], s[3]); cx(s[1], s[2]);
+// Merge an ascending list of 8 keys into c: the same list and evicted as 8
+// cands_insert calls.
+__device__ __forceinline__ void cands_merge8(Cands& c, const float (&s)[TOPK]) {
     float m[8], d[8];
 #pragma unroll
     for (int i = 0; i < TOPK; ++i) {
@@ -213,6 +210,23 @@ __device__ __forceinline__ void cands_insert5(Cands& c, const float (&k)[5]) {
     for (int i = 0; i < TOPK; ++i) c.ts[i] = m[i];
     c.evicted = fminf(c.evicted, fminf(fminf(fmin3(d[0], d[1], d[2]), fmin3(d[3], d[4], d[5])),
                                        fminf(d[6], d[7])));
+}
+__device__ __forceinline__ void cands_insert5(Cands& c, const float (&k)[5]) {
+    const float inf = __int_as_float(0x7f800000);
+    float s[8] = {k[0], k[1], k[2], k[3], k[4], inf, inf, inf};
+    cx(s[0], s[1]); cx(s[3], s[4]); cx(s[2], s[4]);
+    cx(s[2], s[3]); cx(s[0], s[3]); cx(s[0], s[2]);
+    cx(s[1], s[4]); cx(s[1], s[3]); cx(s[1], s[2]);
+    cands_merge8(c, s);
+}
+// Sort 8 keys ascending (a 19-comparator network).
+__device__ __forceinline__ void sort8(float (&s)[8]) {
+    cx(s[0], s[2]); cx(s[1], s[3]); cx(s[4], s[6]); cx(s[5], s[7]);
+    cx(s[0], s[4]); cx(s[1], s[5]); cx(s[2], s[6]); cx(s[3], s[7]);
+    cx(s[0], s[1]); cx(s[2], s[3]); cx(s[4], s[5]); cx(s[6], s[7]);
+    cx(s[2], s[4]); cx(s[3], s[5]);
+    cx(s[1], s[4]); cx(s[3], s[6]);
+    cx(s[1], s[2]); cx(s[3], s[4]); cx(s[5], s[6]);
 }
 
 // Chunk-local keys carry the element's position 0..31 in their 5 low bits;
@@ -873,8 +887,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float best1 = k1[8];
                     cands_insert(cs, fmaxf(cs.best, best1));
                     cs.best = fminf(cs.best, best1);
+                    {
+                        float k1l[TOPK];
 #pragma unroll
-                    for (int p = 0; p < TOPK; ++p) cands_insert(cs, k1[p]);
+                        for (int p = 0; p < TOPK; ++p) k1l[p] = k1[p];
+                        cands_merge8(cs, k1l);  // the other half's ascending list
+                    }
                     if constexpr (kSliced) {
                         // publish this CTA's list of the row, meet the group's other slices,
                         // then merge every slice's list (in slice order, so all slices get
@@ -902,15 +920,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int p = 0; p < kSliceListFloats; ++p) e[t][p] = __ldcg(o + p);
                         }
-                        cands_reset(cs);
+                        // a tree of pairwise merges of the ascending lists, then the
+                        // slices' bests (the smallest is the group's; the other seven,
+                        // sorted, join the list): the list and evicted of inserting every
+                        // key in turn
+                        static_assert(kSlices == 8, "the merge tree assumes 8 slices");
+                        Cands q[4];
 #pragma unroll
-                        for (int t = 0; t < kSlices; ++t) {
-                            cs.evicted = fminf(cs.evicted, e[t][9]);
-                            cands_insert(cs, fmaxf(cs.best, e[t][8]));
-                            cs.best = fminf(cs.best, e[t][8]);
+                        for (int i = 0; i < 4; ++i) {
 #pragma unroll
-                            for (int p = 0; p < TOPK; ++p) cands_insert(cs, e[t][p]);
+                            for (int p = 0; p < TOPK; ++p) q[i].ts[p] = e[2 * i][p];
+                            q[i].evicted = fminf(e[2 * i][9], e[2 * i + 1][9]);
+                            float b[TOPK];
+#pragma unroll
+                            for (int p = 0; p < TOPK; ++p) b[p] = e[2 * i + 1][p];
+                            cands_merge8(q[i], b);
                         }
+                        cands_merge8(q[0], q[1].ts);
+                        q[0].evicted = fminf(q[0].evicted, q[1].evicted);
+                        cands_merge8(q[2], q[3].ts);
+                        q[2].evicted = fminf(q[2].evicted, q[3].evicted);
+                        cands_merge8(q[0], q[2].ts);
+                        q[0].evicted = fminf(q[0].evicted, q[2].evicted);
+                        float bb[kSlices];
+                        float gbest = __int_as_float(0x7f800000);
+#pragma unroll
+                        for (int t = 0; t < kSlices; ++t) gbest = fminf(gbest, e[t][8]);
+#pragma unroll
+                        for (int t = 0; t < kSlices; ++t) bb[t] = e[t][8] == gbest ? __int_as_float(0x7f800000) : e[t][8];
+                        sort8(bb);
+                        cands_merge8(q[0], bb);
+#pragma unroll
+                        for (int p = 0; p < TOPK; ++p) cs.ts[p] = q[0].ts[p];
+                        cs.evicted = q[0].evicted;
+                        cs.best = gbest;
                     }
                     cands_insert(cs, cs.best);  // the best heads the candidate list
                     const float wthr = cs.best + key_slack(cs.best) + twoE;
