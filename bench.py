@@ -79,8 +79,8 @@ MOSHI_DELAYS = [0, 1, 1, 1, 1, 1, 1, 1]   # acoustic delay 1 (the final model's)
 # summary that records it; the bench scales it by the units of a launch. None: not captured.
 NCU_TRAFFIC_PER_UNIT = {
     "k_embed_sum": (48_927, "profiles/k_embed_sum_moshi_input.md"),        # per step
-    "k_encode_tc/f32": (2_488, "profiles/k_encode_tc_offline_batch_fp32.md"),  # per fp32 frame
-    "k_encode_tc/bf16": (1_163, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
+    "k_encode_tc/f32": (2_493, "profiles/k_encode_tc_offline_batch_fp32.md"),  # per fp32 frame
+    "k_encode_tc/bf16": (1_159, "profiles/k_encode_tc_bulk_tokenization.md"),  # per bf16 frame
     "k_decode": (1_987, "profiles/k_decode_decode_heavy.md"),              # per frame
 }
 
