@@ -132,6 +132,11 @@ __device__ __forceinline__ void issue_chunk(const WideArgs& a, float* buf, int c
 template <int U, int V>
 __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
     constexpr int KS = 16 * V;
+    // global loads per thread issued together: many for groups of more than 16
+    // frames (fewer for the largest thread tile, whose scoring registers leave less
+    // room); 4 for the smallest steps, which have few loads to batch and are
+    // measured faster with the smaller register footprint
+    constexpr int kBatch = U == 1 ? 4 : (U * V >= 16 ? 8 : 16);
     extern __shared__ __align__(16) float smem_w[];
     // c_buf0 | r_s | c_buf1 ; the projection stages its operands over r_s .. c_buf1
     auto cbuf = [&](int c) { return smem_w + ((c & 1) ? (KS + FG) * RSTRIDE : 0); };
@@ -193,10 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
             for (int j0 = 0; j0 < kDin; j0 += JC) {
                 __syncthreads();
                 const int nz = F * J4, nt = (F + nd) * J4;
-                for (int e0 = tid; e0 < nt; e0 += 4 * kThreads) {
-                    float4 v[4];
+                for (int e0 = tid; e0 < nt; e0 += kBatch * kThreads) {
+                    float4 v[kBatch];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < kBatch; ++u) {
                         const int e = e0 + u * kThreads;
                         if (e < nz)
                             v[u] = load_latent4(a.z, a.dtype, (int64_t)frame_s[e / J4] * kDin + j0 + 4 * (e % J4));
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
                                 a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
                     }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < kBatch; ++u) {
                         const int e = e0 + u * kThreads;
                         if (e < nt) {
                             float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
@@ -318,19 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
                 cp_async_wait_all();
                 return;
             }
-            // winners: minimum over the group's S slots of each frame (loads in batches of 4)
+            // winners: minimum over the group's S slots of each frame (loads in batches of
+            // kBatch, all in flight together)
             {
                 unsigned long long m = ~0ull;
                 if (rf < F)
-                    for (int s0 = rsub; s0 < S; s0 += 4 * tpf) {
-                        unsigned long long v[4];
+                    for (int s0 = rsub; s0 < S; s0 += kBatch * tpf) {
+                        unsigned long long v[kBatch];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < kBatch; ++u) {
                             const int sl = s0 + u * tpf;
                             v[u] = sl < S ? __ldcg(part + (size_t)rf * S + sl) : ~0ull;
                         }
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) m = umin64(m, v[u]);
+                        for (int u = 0; u < kBatch; ++u) m = umin64(m, v[u]);
                     }
                 for (int o = tpf >> 1; o > 0; o >>= 1) m = umin64(m, __shfl_xor_sync(0xffffffffu, m, o));
                 if (rsub == 0 && rf < F) {
@@ -349,17 +355,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
             __syncthreads();
             // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
             if (l < a.n_q - 1 && (l >= 1 || a.variant == 1)) {
+                // the winners' rows in batches of kBatch loads per thread, all in flight
+                // before the subtractions
                 const float* book = a.C32 + (size_t)l * kK * kD;
-                for (int e = tid; e < F * (kD / 4); e += kThreads) {
-                    const int f = e / (kD / 4), i4 = e % (kD / 4);
-                    const float4 cw = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[f] * kD) + i4);
-                    float4* r = reinterpret_cast<float4*>(r_s + f * RSTRIDE + 4 * i4);
-                    float4 v = *r;
-                    v.x -= cw.x;
-                    v.y -= cw.y;
-                    v.z -= cw.z;
-                    v.w -= cw.w;
-                    *r = v;
+                const int ne = F * (kD / 4);
+                for (int e0 = tid; e0 < ne; e0 += kBatch * kThreads) {
+                    float4 cw[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < ne)
+                            cw[u] = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[e / (kD / 4)] * kD) +
+                                          e % (kD / 4));
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < ne) {
+                            float4* r = reinterpret_cast<float4*>(r_s + (e / (kD / 4)) * RSTRIDE + 4 * (e % (kD / 4)));
+                            float4 v = *r;
+                            v.x -= cw[u].x;
+                            v.y -= cw[u].y;
+                            v.z -= cw[u].z;
+                            v.w -= cw[u].w;
+                            *r = v;
+                        }
+                    }
                 }
             }
         }
