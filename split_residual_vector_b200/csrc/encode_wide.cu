@@ -100,7 +100,7 @@ struct WideArgs {
     unsigned long long* stats;
     const void* z;
     int dtype, B, n_q, variant;
-    int groups, S, per_k, jc;
+    int groups, S, per_k, jc, fb;
     int16_t* codes;
     float* y;                       // [B][256] projection exchange
     unsigned* bars;                 // [kWideMaxGroups][kWideBarStride] barrier words
@@ -172,17 +172,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
         __syncthreads();
         issue_chunk<KS>(a, cbuf(0), 0, nch, k_lo, k_hi);
 
-        // ---- y = W_in . z for output dimensions [d0, d1) of every frame of the group,
-        //      each output a sequential FMA chain over j (the full scan's order). The
-        //      latents and W_in rows are staged in passes of JC columns (row stride
-        //      JC + 1: conflict-free column reads), with batched vector loads.
+        // ---- y = W_in . z, the group's frames x 256 outputs split over its S CTAs as
+        //      fb frame blocks x S / fb output blocks: this CTA computes frames
+        //      [fb0, fb1) x outputs [d0, d1), each output a sequential FMA chain over j
+        //      (the full scan's order). The latents and W_in rows are staged in passes of
+        //      JC columns (row stride JC + 1: conflict-free column reads), with batched
+        //      vector loads.
         {
-            const int per = (kD + S - 1) / S;
-            const int d0 = min(kD, member * per), d1 = min(kD, d0 + per), nd = d1 - d0;
-            const int items = F * nd;
+            const int OB = S / a.fb;
+            const int fpb = (F + a.fb - 1) / a.fb, opb = (kD + OB - 1) / OB;
+            const int fb0 = min(F, (member / OB) * fpb), fb1 = min(F, fb0 + fpb), nf = fb1 - fb0;
+            const int d0 = min(kD, (member % OB) * opb), d1 = min(kD, d0 + opb), nd = d1 - d0;
+            const int items = nf * nd;
             const int JC = a.jc, JS = JC + 1, J4 = JC / 4;
-            float* z_s = r_s;             // [F][JS]
-            float* w_s = r_s + F * JS;    // [nd][JS]
+            float* z_s = r_s;             // [nf][JS]
+            float* w_s = r_s + nf * JS;   // [nd][JS]
             const int nq_items = (items + kThreads - 1) / kThreads;  // uniform over the CTA
             int zo[kProjItems], wo[kProjItems];
             bool act[kProjItems];
@@ -197,14 +201,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
             }
             for (int j0 = 0; j0 < kDin; j0 += JC) {
                 __syncthreads();
-                const int nz = F * J4, nt = (F + nd) * J4;
+                const int nz = nf * J4, nt = (nf + nd) * J4;
                 for (int e0 = tid; e0 < nt; e0 += kBatch * kThreads) {
                     float4 v[kBatch];
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         const int e = e0 + u * kThreads;
                         if (e < nz)
-                            v[u] = load_latent4(a.z, a.dtype, (int64_t)frame_s[e / J4] * kDin + j0 + 4 * (e % J4));
+                            v[u] = load_latent4(a.z, a.dtype, (int64_t)frame_s[fb0 + e / J4] * kDin + j0 + 4 * (e % J4));
                         else if (e < nt)
                             v[u] = __ldg(reinterpret_cast<const float4*>(
                                 a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
             for (int q = 0; q < kProjItems; ++q)
                 if (act[q]) {
                     const int it = tid + q * kThreads;
-                    a.y[(size_t)(f0 + it / nd) * kD + d0 + it % nd] = acc[q];
+                    a.y[(size_t)(f0 + fb0 + it / nd) * kD + d0 + it % nd] = acc[q];
                 }
         }
         ++episode;
@@ -429,13 +433,24 @@ WidePlan plan_encode_wide(int B, int num_sms) {
     const int fmax = B < FG ? B : FG;
     p.U = fmax <= 16 ? 1 : fmax <= 32 ? 2 : 4;
     p.V = per_k <= 16 ? 1 : per_k <= 32 ? 2 : 4;
-    // projection: at most kProjItems outputs per thread, operands staged in
-    // chunks of jc latent columns over the r tile and the second codeword buffer
-    const int nd = (kD + p.S - 1) / p.S;
-    if (fmax * nd > kProjItems * kThreads) return p;
+    // projection: the frames x outputs of a group split into fb frame blocks x
+    // S / fb output blocks (fb a power of two dividing S, at most the frames),
+    // chosen to stage the fewest rows (latents + W_in) per CTA; at most kProjItems
+    // outputs per thread, operands staged in chunks of jc latent columns over the r
+    // tile and the second codeword buffer
+    int best_rows = 1 << 30;
+    for (int fb = 1; fb <= fmax && p.S % fb == 0; fb *= 2) {
+        const int rows = (fmax + fb - 1) / fb + (kD + p.S / fb - 1) / (p.S / fb);
+        if (rows < best_rows) {
+            best_rows = rows;
+            p.fb = fb;
+        }
+    }
+    const int fpb = (fmax + p.fb - 1) / p.fb, opb = (kD + p.S / p.fb - 1) / (p.S / p.fb);
+    if (fpb * opb > kProjItems * kThreads) return p;
     const int region = (FG + 16 * p.V) * RSTRIDE;
     for (int jc = kDin; jc >= 16; jc >>= 1)
-        if ((fmax + nd) * (jc + 1) <= region) {
+        if ((fpb + opb) * (jc + 1) <= region) {
             p.jc = jc;
             break;
         }
@@ -485,6 +500,7 @@ cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z
     a.S = p.S;
     a.per_k = p.per_k;
     a.jc = p.jc;
+    a.fb = p.fb;
     a.codes = codes;
     a.y = t.wide_y;
     a.bars = t.wide_bars;

@@ -100,6 +100,7 @@ struct WidePlan {
     int grid = 0;      // groups * S (<= SM count: every CTA resident at once)
     int U = 0, V = 0;  // thread tile: 16U frames x 16V codewords
     int jc = 0;        // projection: latent columns staged per pass
+    int fb = 1;        // projection: frame blocks per group (S / fb output blocks)
     int smem = 0;      // dynamic shared memory bytes
 };
 WidePlan plan_encode_wide(int B, int num_sms);
