@@ -268,6 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
                 __syncthreads();  // chunk c landed; chunk c - 1 consumed; r_s up to date
                 if (c + 1 < total) issue_chunk<KS>(a, cbuf(c + 1), c + 1, nch, k_lo, k_hi);
                 const float* c_s = cbuf(c);
+                // the chunk's ||c||^2, loaded before the dot products so that their latency
+                // is hidden (for the widest codeword tile after them: it was measured
+                // slower there, its accumulators leave no registers to spare)
+                float cnv[V];
+                if constexpr (V <= 2) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) cnv[v] = tk + 16 * v < nk ? __ldg(cn + kc + tk + 16 * v) : 0.f;
+                }
                 float acc[U][V][4];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
@@ -298,11 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_encode_wide(WideArgs a) {
                 for (int v = 0; v < V; ++v) {
                     const int k = tk + 16 * v;
                     if (k < nk) {
-                        const float cnk = __ldg(cn + kc + k);
+                        if constexpr (V > 2) cnv[v] = __ldg(cn + kc + k);
 #pragma unroll
                         for (int u = 0; u < U; ++u) {
                             const float dot = (acc[u][v][0] + acc[u][v][1]) + (acc[u][v][2] + acc[u][v][3]);
-                            mk[u] = umin64(mk[u], pack_key(fmaf(-2.f, dot, cnk), kc + k));
+                            mk[u] = umin64(mk[u], pack_key(fmaf(-2.f, dot, cnv[v]), kc + k));
                         }
                     }
                 }
