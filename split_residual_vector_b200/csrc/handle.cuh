@@ -19,11 +19,9 @@ constexpr int kQ = 8;         // codebooks: 0 semantic, 1..7 acoustic
 // list cannot overflow).
 constexpr int64_t kRescanCapacity = 1 << 20;
 
-// Largest streaming step the latency (wide) encoder takes; larger steps go to
-// the tensor-core encoder. Measured per-call latency on B200: 54 us at 1 frame,
-// 121 us at 128, 318 us at 768, 392 us at 1024; the tensor-core encoder takes
-// 290-380 us plus, from a few hundred frames up, the float32 re-scan of its
-// (usually one or two) uncertified frames, ~400 us for a single frame.
+// Largest batch the latency (wide) encoder takes: streaming steps up to
+// kSlicedMinFrames - 1 frames, and the float32 re-encode of the frames the batch
+// tensor-core encoder could not certify, 1024 at a time.
 constexpr int kWideMaxFrames = 1024;
 constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
 constexpr int kWideMaxGroups = 64;    // group barriers (the last one is the wait self-test's)
@@ -40,7 +38,10 @@ constexpr int kSliceBarBase = 32;
 constexpr int kSliceListFloats = 10;  // per row: 8 candidate keys, best, evicted
 // Streaming steps of at least this many frames take the sliced tensor-core
 // encoder (when its CTAs fit the device); smaller ones the float32 latency encoder.
-constexpr int kSlicedMinFrames = 512;
+// Measured per step on B200: the latency encoder 52 us at 1 frame, 105 us at 128,
+// 136 us at 256, but 211-219 us from 320 to 511 frames (five groups and more);
+// the sliced encoder 207-209 us from 256 to 511 frames, 215 us at 1024.
+constexpr int kSlicedMinFrames = 257;
 
 struct Tables {
     int num_sms = 148;            // SMs of the handle's device (grid sizes)

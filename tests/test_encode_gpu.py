@@ -164,15 +164,15 @@ def test_streaming_step(batch):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_small_streaming_steps_equal_the_full_scan(dtype):
-    """Steps under 512 frames run the latency encoder, whose scores are the float32 full
+    """Steps of at most 256 frames run the latency encoder, whose scores are the float32 full
     scan's (same sums in the same order): every code equals encode_scan's, near ties
-    included. Sizes span one to eight frame groups, ragged group tails and every thread-tile
+    included. Sizes span one to four frame groups, ragged group tails and every thread-tile
     shape."""
     model, frames = synth.streaming_step(1024, calls=1)
     q = quantizer(model)
     z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
     zd = to_device(np.ascontiguousarray(z))
-    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 500, 511)
+    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 200, 255, 256)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         scan = q.encode_scan(zd[:b]).cpu().numpy()
@@ -184,7 +184,7 @@ def test_small_streaming_steps_equal_the_full_scan(dtype):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_sliced_streaming_steps_match_the_oracle(dtype):
-    """Steps of 512 frames and more run the codebook-sliced tensor-core encoder (8 CTAs per
+    """Steps of more than 256 frames run the codebook-sliced tensor-core encoder (8 CTAs per
     128-frame group, candidate lists exchanged through global memory): codes equal the
     oracle's outside near-ties and the batch tensor-core encoder's on every other frame,
     for full and ragged groups, up to the 18 groups that fit the device at once."""
@@ -195,7 +195,7 @@ def test_sliced_streaming_steps_match_the_oracle(dtype):
     ref, db, ds = oracle.encode(z, model.W_in, model.C)
     near = oracle.near_tie(db, ds)
     enc0, _ = q.stats()
-    sizes = (512, 513, 700, 896, 1000, 1024, 2304)
+    sizes = (257, 300, 384, 511, 512, 513, 700, 896, 1000, 1024, 2304)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         assert_codes_match(step, ref[:b], db[:b], ds[:b], f"sliced step B={b}")
