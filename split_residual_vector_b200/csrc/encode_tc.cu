@@ -10,10 +10,10 @@
 //      the whole level chain: it never leaves the SM.
 //   2. for each codebook l = 0 (semantic, on y) and 1..7 (acoustic, on r):
 //      candidate half-scores ||c||^2 / 2 - bf16(r) . bf16(c) for all 2048
-//      codewords as 8 tcgen05 GEMM tiles [128 x 256] x [256 x 256]. Each tile
-//      starts with one K = 16 step that writes ||c||^2 / 2 into the accumulator
-//      (A = ones, B = the norm's three exact bf16 parts) and continues with A =
-//      -bf16(r), so the epilogue reads the half-score directly (codebook tiles
+//      codewords as 8 tcgen05 GEMM tiles [128 x 256] x [256 x 256] with A =
+//      -bf16(r). Each tile ends with one K = 16 step that adds ||c||^2 / 2 into
+//      the accumulator (A = ones, B = the norm's three exact bf16 parts), so the
+//      epilogue reads the half-score directly (codebook tiles
 //      streamed by TMA into a shared-memory ring, one 256-row box per stage;
 //      the accumulator is TMEM columns [256, 512), which the epilogue copies
 //      into registers at once so that the next tile's MMAs overlap its scan).
@@ -26,14 +26,16 @@
 //      (||c||^2 - 2 r.c with r read from TMEM and c from the float32
 //      codebook); a single candidate needs no re-score. If the top-8 cannot be
 //      certified the frame is queued for a float32 re-encode (the wide encoder,
-//      in list mode, after this kernel).
+//      in list mode, after this kernel); the sliced streaming form instead scans
+//      that row exactly in float32 inside the kernel.
 //   4. acoustic levels: r -= c_win in TMEM, and bf16(r) is written into the
 //      shared-memory A operand of the next level.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues the MMAs (one thread), warps 2..9 are the epilogue: the two warps of a
-// TMEM lane quarter (frame rows 32q .. 32q + 31) split each score tile's
-// columns and the residual's dimensions between them. The semantic level (0)
+// Warp roles (384 threads, three warpgroups): warp 0 issues TMA loads, warp 1
+// allocates TMEM and issues the MMAs (one thread each), warps 2 and 3 idle;
+// warps 4..11 are the epilogue: the two warps of a TMEM lane quarter (frame rows
+// 32q .. 32q + 31) split each score tile's columns and the residual's
+// dimensions between them. The semantic level (0)
 // and acoustic level 1 share the A operand bf16(y), so the tensor core runs
 // from level 0 into level 1 while the epilogue re-scores level 0.
 #include <cuda.h>

@@ -15,9 +15,11 @@
 // reduces the S slots of each frame -- so the lowest score wins and ties go to
 // the lowest index -- and applies the same residual update to its own copy of
 // r in shared memory: one barrier per level. The projection y = W_in . z is
-// split by output dimension over the group's CTAs and exchanged through global
-// memory behind one more barrier. Every sum is taken in the float32 full
-// scan's order, so the codes are the ones mimi_rvq_encode_scan returns.
+// split over the group's CTAs as frame blocks x output blocks and exchanged
+// through global memory behind one more barrier. Every sum is taken in the
+// float32 full scan's order, so the codes are the ones mimi_rvq_encode_scan
+// returns. It serves streaming steps of up to 256 frames and the re-encode of
+// the frames the batch tensor-core encoder could not certify.
 //
 // Codeword chunks are double-buffered with cp.async; the next level's first
 // chunk does not depend on the winners, so its copy overlaps the barrier.
