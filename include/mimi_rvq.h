@@ -206,7 +206,9 @@ int mimi_rvq_wait_selftest(mimi_rvq_t h, int which, struct CUstream_st *stream);
 /*
  * Counters since create (synchronises `stream`): frames encoded, and frames
  * whose bf16 candidate pass could not certify its candidate set at some level
- * and were re-encoded by the full float32 scan. Either pointer may be NULL.
+ * and were resolved in float32 instead (re-encoded by the full scan after a
+ * batch encode; the row scanned exactly inside the kernel in a sliced
+ * streaming step). Either pointer may be NULL.
  */
 int mimi_rvq_stats(mimi_rvq_t h, struct CUstream_st *stream, int64_t *frames_encoded,
                    int64_t *frames_rescanned);

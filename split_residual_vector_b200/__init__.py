@@ -251,7 +251,8 @@ class Quantizer:
         return int(library().mimi_rvq_get_error(self._h, _stream(stream)))
 
     def stats(self, stream=None):
-        """(frames encoded, frames re-encoded by the float32 full scan) since create."""
+        """(frames encoded, frames whose candidates could not be certified and were resolved in
+        float32: re-encoded after a batch encode, scanned exactly in a sliced step) since create."""
         a, b = ctypes.c_int64(), ctypes.c_int64()
         _check(library().mimi_rvq_stats(self._h, _stream(stream), ctypes.byref(a),
                                         ctypes.byref(b)), "mimi_rvq_stats")
