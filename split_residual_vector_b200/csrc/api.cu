@@ -63,6 +63,21 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x 256 rows
 // (32 KiB: one stage of the tensor-core encoder's ring), 128-byte swizzle: the
 // layout the UMMA shared-memory descriptors expect.
+// 2-D fp32 tensor [rows][cols] (row-major), boxes of 32 columns x box_rows rows
+// (one 128-byte row per codeword), 128-byte swizzle: the cluster encoder's slabs.
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {32, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -189,6 +204,7 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     if (s) cudaStreamDestroy(s);
     if (e == cudaSuccess) e = mimi::encode_tc_configure();
     if (e == cudaSuccess) e = mimi::encode_wide_configure();
+    if (e == cudaSuccess) e = mimi::encode_cluster_configure(t);
     if (e != cudaSuccess) {
         free_tables(t);
         delete h;
@@ -201,6 +217,9 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
         delete h;
         return MIMI_RVQ_ECUDA;
     }
+    // the cluster form needs its slab maps; a size without one stays off
+    if (!make_tmap_f32(&t.tm_C32_8, t.C32, (uint64_t)kQ * kK, kD, kK / 8)) t.cl_max8 = 0;
+    if (!make_tmap_f32(&t.tm_C32_16, t.C32, (uint64_t)kQ * kK, kD, kK / 16)) t.cl_max16 = 0;
     *out = h;
     return MIMI_RVQ_OK;
 }
@@ -247,6 +266,14 @@ int mimi_rvq_encode_step_ex(mimi_rvq_t h, const void* frames, int dtype, int B, 
     if (!h || B < 0) return MIMI_RVQ_EINVAL;
     if (dtype != MIMI_RVQ_F32 && dtype != MIMI_RVQ_BF16) return MIMI_RVQ_EINVAL;
     if (n_q < 1 || n_q > kQ || (variant != 0 && variant != 1)) return MIMI_RVQ_EINVAL;
+    const mimi::ClusterPlan cp = mimi::plan_encode_cluster(h->t, B);
+    if (cp.ok) {
+        // float32 latency encode on thread-block clusters
+        const int c = check_common(h, frames, codes, B);
+        if (c <= 0) return c;
+        return from_cuda(
+            mimi::launch_encode_cluster(h->t, cp, frames, dtype, B, n_q, variant, codes, stream));
+    }
     if (B >= mimi::kSlicedMinFrames && mimi::sliced_fits(B, h->num_sms)) {
         // codebook-sliced tensor-core encode (rows it cannot certify take an exact
         // float32 scan inside the kernel: one launch)

@@ -1,0 +1,442 @@
+// encode_cluster.cu -- latency encode of a streaming step on thread-block clusters.
+//
+// The frames of a step are cut into blocks of at most 32, one per cluster of CS
+// CTAs (16 where the device co-schedules at least as many CTAs that way, else
+// 8). CTA `rank` of a cluster owns codewords [rank * K / CS, (rank + 1) * K / CS)
+// of every codebook and scores them against all frames of its block on the CUDA
+// cores, in float32 and in the full scan's order:
+//
+//   score(f, k) = ||c_k||^2 - 2 r_f . c_k      (4 partial sums, as the full scan)
+//
+// Per level each CTA reduces its keys (order-preserving score bits, codeword
+// index) per frame into its own shared memory; one cluster barrier closes the
+// level, and every CTA then reads the CS minima of each frame through
+// distributed shared memory, so all pick the same winner (lowest score, ties to
+// the lowest index) and apply the same update to their own copy of r. The
+// projection y = W_in . z is split over the cluster's CTAs by output dimension
+// and gathered the same way. The codes are the ones mimi_rvq_encode_scan
+// returns.
+//
+// Against the group form of encode_wide.cu (groups of CTAs meeting at barriers
+// in global memory): a cluster barrier is a hardware barrier, the minima cross
+// no L2 round trips, and a CTA updates r for the few frames of its cluster
+// only. Clusters never wait on one another, so the launch needs no
+// co-residency guarantee and leaves no state behind (graph replays and
+// concurrent streams need no reset).
+//
+// Scoring is bound by shared-memory operand traffic, so the thread tile is
+// chosen for it: the four lanes w = 0..3 of a lane quad each keep one of the
+// four partial sums (dimensions i + w, i stepping by 4) of U frames x V
+// codewords, reading their operands with 32-bit loads that hit 32 distinct
+// banks (a warp's 8 quads take 8 consecutive codewords); the partials are
+// combined at the end of the level by two shuffles, (p0 + p1) + (p2 + p3),
+// the scan's order. The CTA's codewords arrive by TMA as slabs of 32
+// dimensions (one 128-byte row per codeword, 128-byte swizzle) through a
+// 4-stage ring; one thread refills a stage once every warp is done with it.
+#include "latency_common.cuh"
+
+namespace mimi {
+namespace {
+
+using lat::kProjItems;
+using lat::kThreads;
+using lat::load_latent4;
+using lat::pack_key;
+using lat::RSTRIDE;
+using lat::umin64;
+
+constexpr int kSlabDims = 32;                        // dimensions per slab (128 bytes per codeword)
+constexpr int kSlabsPerLevel = kD / kSlabDims;       // 8
+constexpr int NST = 4;                               // slab stages
+constexpr int kMaxSlice = kK / 8;                    // codewords per CTA in clusters of 8
+constexpr int STAGE_BYTES = kMaxSlice * 128;         // 32 KiB
+constexpr int YSTRIDE = 32;                          // row stride (floats) of the projection block
+constexpr int R_OFF = NST * STAGE_BYTES;             // bytes: r rows
+constexpr int Y_OFF = R_OFF + kClusterMaxBlock * RSTRIDE * 4;      // projection block
+constexpr int MK_OFF = Y_OFF + kClusterMaxBlock * YSTRIDE * 4;     // [2][block] minimum keys
+constexpr int WIN_OFF = MK_OFF + 2 * kClusterMaxBlock * 8;         // [block] winners
+constexpr int BAR_OFF = WIN_OFF + kClusterMaxBlock * 4;            // [NST] slab barriers
+constexpr int ABORT_OFF = BAR_OFF + NST * 8;
+constexpr int RED_OFF = ABORT_OFF + 16;                            // [8 warps][16] per-warp minima
+constexpr int SMEM_BYTES = RED_OFF + 8 * 16 * 8 + 1024;  // + alignment of the swizzled stages
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(BAR_OFF % 8 == 0 && MK_OFF % 8 == 0 && RED_OFF % 8 == 0, "alignment");
+// the projection stages F + kD / CS rows of all kDin + 1 columns over the slab stages and the
+// r rows, before either is in use
+static_assert((kClusterMaxBlock + kD / 8) * (kDin + 1) * 4 <= Y_OFF, "projection staging fits");
+
+struct ClusterArgs {
+    const float* C32;
+    const float* Win32;
+    const float* cnorm;
+    int* err;
+    unsigned long long* stats;
+    const void* z;
+    int dtype, B, n_q, variant;
+    int cs;   // CTAs per cluster
+    int fc;   // frames per cluster (the last cluster may have fewer)
+    int16_t* codes;
+};
+
+// Thread tile U frames x V codewords per lane quad; warps split as WF (frame
+// blocks of U) x WC (codeword blocks of 8V), WC = (K / CS) / (8V).
+template <int U, int V>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_encode_cluster(const __grid_constant__ CUtensorMap tm_C32, ClusterArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float* r_s = reinterpret_cast<float*>(sm + R_OFF);
+    float* y_s = reinterpret_cast<float*>(sm + Y_OFF);
+    unsigned long long* mk_s = reinterpret_cast<unsigned long long*>(sm + MK_OFF);
+    int* win_s = reinterpret_cast<int*>(sm + WIN_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + BAR_OFF);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + ABORT_OFF);
+    unsigned long long* red_s = reinterpret_cast<unsigned long long*>(sm + RED_OFF);
+
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int g = lane >> 2, w = lane & 3;
+    const int cs = a.cs;
+    const int rank = (int)cluster_ctarank();
+    const int f0 = (blockIdx.x / cs) * a.fc;
+    const int F = min(a.fc, a.B - f0);  // >= 1: the plan launches no empty cluster
+    const int slice = kK / cs;
+    const int WC = slice / (8 * V);
+    const int wf = wid / WC, wc = wid % WC;
+    const int k_base = rank * slice;
+    const int DO = kD / cs;             // projection outputs of this CTA: [rank * DO, rank * DO + DO)
+    const int total = a.n_q * kSlabsPerLevel;
+    const uint32_t stage_tx = (uint32_t)slice * 128u;
+
+    // slab s: dimensions [32 (s % 8), + 32) of this CTA's codewords of level s / 8
+    auto issue = [&](int s) {
+        uint64_t* bar = &full[s % NST];
+        mbar_arrive_expect_tx(bar, stage_tx);
+        tma_load_2d(sm + (s % NST) * STAGE_BYTES, &tm_C32, bar, (s % kSlabsPerLevel) * kSlabDims,
+                    (s / kSlabsPerLevel) * kK + k_base);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---- y = W_in . z for the cluster's F frames x this CTA's DO outputs, each a
+    //      sequential FMA chain over j (the full scan's order); latents and W_in rows
+    //      staged whole (every load in flight at once) over the slab stages and r rows
+    {
+        const int d0 = rank * DO;
+        const int items = F * DO;
+        constexpr int JC = kDin, JS = JC + 1, J4 = JC / 4;
+        float* z_s = reinterpret_cast<float*>(sm);   // [F][JS]
+        float* w_s = z_s + F * JS;                   // [DO][JS]
+        const int nq_items = (items + kThreads - 1) / kThreads;  // uniform over the CTA
+        int zo[kProjItems], wo[kProjItems];
+        float acc[kProjItems];
+#pragma unroll
+        for (int q = 0; q < kProjItems; ++q) {
+            const int it = tid + q * kThreads;
+            const bool act = it < items;
+            zo[q] = act ? (it / DO) * JS : 0;
+            wo[q] = act ? (it % DO) * JS : 0;
+            acc[q] = 0.f;
+        }
+        for (int j0 = 0; j0 < kDin; j0 += JC) {
+            __syncthreads();
+            const int nz = F * J4, nt = (F + DO) * J4;
+            for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
+                float4 v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * kThreads;
+                    if (e < nz)
+                        v[u] = load_latent4(a.z, a.dtype, (int64_t)(f0 + e / J4) * kDin + j0 + 4 * (e % J4));
+                    else if (e < nt)
+                        v[u] = __ldg(reinterpret_cast<const float4*>(
+                            a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * kThreads;
+                    if (e < nt) {
+                        float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
+                        d[0] = v[u].x;
+                        d[1] = v[u].y;
+                        d[2] = v[u].z;
+                        d[3] = v[u].w;
+                    }
+                }
+            }
+            __syncthreads();
+            lat::proj_chain_any(nq_items, z_s, w_s, zo, wo, acc, JC);
+        }
+#pragma unroll
+        for (int q = 0; q < kProjItems; ++q) {
+            const int it = tid + q * kThreads;
+            if (it < items) y_s[(it / DO) * YSTRIDE + it % DO] = acc[q];
+        }
+    }
+    __syncthreads();  // the staging is read: the stages take the first slabs
+    if (tid == 0)
+        for (int s = 0; s < NST && s < total; ++s) issue(s);
+    cluster_sync();  // every CTA's projection block is written
+
+    // r = y, gathered from the cluster's CTAs; the rows past F up to the thread
+    // tile's end are zero (scored, never published)
+    const int rows = (8 / WC) * U;
+    for (int e = tid; e < rows * (kD / 4); e += kThreads) {
+        const int f = e >> 6, d = 4 * (e & 63);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (f < F) v = ld_cluster_f4(cluster_map(smem_u32(y_s + f * YSTRIDE + d % DO), (uint32_t)(d / DO)));
+        *reinterpret_cast<float4*>(r_s + f * RSTRIDE + d) = v;
+    }
+    __syncthreads();
+
+    // this lane's codewords (row within the CTA's slice: cw0 + 8v) and frames (fr0 + u)
+    const int cw0 = wc * 8 * V + g;
+    const int fr0 = wf * U;
+    int s = 0;  // slab index over all levels
+    for (int l = 0; l < a.n_q; ++l) {
+        // minima by level parity: a slot is rewritten two levels later, after the
+        // barrier that every CTA reaches only once it has read it
+        unsigned long long* mk = mk_s + (l & 1) * kClusterMaxBlock;
+        float cnv[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) cnv[v] = __ldg(a.cnorm + (size_t)l * kK + k_base + cw0 + 8 * v);
+        float acc[U][V];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
+        for (int j = 0; j < kSlabsPerLevel; ++j, ++s) {
+            mbar_wait(&full[s % NST], (uint32_t)(s / NST) & 1u, abort, a.err);
+            // codeword row cw0 + 8v of the stage: 128 bytes, 16-byte unit x at x ^ (row & 7),
+            // and row & 7 = g
+            const uint8_t* cb = sm + (s % NST) * STAGE_BYTES + cw0 * 128 + 4 * w;
+            const float* rb = r_s + fr0 * RSTRIDE + j * kSlabDims + w;
+#pragma unroll
+            for (int i = 0; i < kSlabDims; i += 4) {
+                const int off = ((i >> 2) ^ g) << 4;
+                float cv[V], rv[U];
+#pragma unroll
+                for (int v = 0; v < V; ++v) cv[v] = *reinterpret_cast<const float*>(cb + v * 1024 + off);
+#pragma unroll
+                for (int u = 0; u < U; ++u) rv[u] = rb[u * RSTRIDE + i];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[u][v] = fmaf(rv[u], cv[v], acc[u][v]);
+            }
+            __syncthreads();  // every warp is done with the stage
+            if (tid == 0 && s + NST < total) issue(s + NST);
+        }
+        // dot = (p0 + p1) + (p2 + p3) across the quad, then the minimum key per frame over
+        // the warp's codewords and one shared atomic per warp and frame
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            unsigned long long best = ~0ull;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                float p = acc[u][v];
+                p = p + __shfl_xor_sync(0xffffffffu, p, 1);
+                p = p + __shfl_xor_sync(0xffffffffu, p, 2);
+                best = umin64(best, pack_key(fmaf(-2.f, p, cnv[v]), k_base + cw0 + 8 * v));
+            }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) best = umin64(best, __shfl_xor_sync(0xffffffffu, best, o));
+            if (lane == 0) red_s[wid * 16 + u] = best;
+        }
+        __syncthreads();
+        // frame f: the minimum over the WC warps that scored its codewords
+        if (tid < F) {
+            const int fw = (tid / U) * WC, fu = tid % U;
+            unsigned long long m = red_s[fw * 16 + fu];
+            for (int c = 1; c < WC; ++c) m = umin64(m, red_s[(fw + c) * 16 + fu]);
+            mk[tid] = m;
+        }
+        cluster_sync();  // every CTA's minima of this level are in its shared memory
+        // winners: the minimum over the cluster's CTAs of each frame
+        if (tid < F) {
+            const uint32_t addr = smem_u32(mk + tid);
+            unsigned long long m[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) m[r] = r < cs ? ld_cluster_u64(cluster_map(addr, (uint32_t)r)) : ~0ull;
+#pragma unroll
+            for (int r = 1; r < 16; ++r) m[0] = umin64(m[0], m[r]);
+            int wn = (int)(uint32_t)m[0];
+            if (wn < 0 || wn >= kK) wn = 0;  // only reachable with NaN / Inf inputs
+            win_s[tid] = wn;
+            if (rank == 0) a.codes[(size_t)(f0 + tid) * a.n_q + l] = (int16_t)wn;
+        }
+        if (l == a.n_q - 1) break;
+        __syncthreads();
+        // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
+        if (l >= 1 || a.variant == 1) {
+            const float* book = a.C32 + (size_t)l * kK * kD;
+            const int ne = F * (kD / 4);
+            for (int e0 = tid; e0 < ne; e0 += 8 * kThreads) {
+                float4 cw[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int e = e0 + u * kThreads;
+                    if (e < ne) cw[u] = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[e >> 6] * kD) + (e & 63));
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int e = e0 + u * kThreads;
+                    if (e < ne) {
+                        float4* r = reinterpret_cast<float4*>(r_s + (e >> 6) * RSTRIDE + 4 * (e & 63));
+                        float4 v = *r;
+                        v.x -= cw[u].x;
+                        v.y -= cw[u].y;
+                        v.z -= cw[u].z;
+                        v.w -= cw[u].w;
+                        *r = v;
+                    }
+                }
+            }
+        }
+        __syncthreads();  // r updated before the next level's scores
+    }
+    if (blockIdx.x == 0 && tid == 0) atomicAdd(&a.stats[0], (unsigned long long)a.B);
+    cluster_sync();  // no CTA leaves while another may still read its shared memory
+}
+
+// The thread tiles built, as (U, V): V = 4 (one warp per frame block: rows = U
+// with clusters of 8) for small blocks, V = 8 (two or four warps per frame
+// block) for large ones, so that every frame count from 1 to 32 has a tile with
+// little padding. A plan takes the cheapest by the cost model below.
+struct Tile {
+    int U, V;
+    const void* kernel;
+};
+template <int U, int V>
+Tile tile() {
+    return {U, V, reinterpret_cast<const void*>(k_encode_cluster<U, V>)};
+}
+const Tile kTiles[] = {tile<1, 4>(), tile<2, 4>(), tile<3, 4>(),  tile<4, 4>(),  tile<6, 4>(),
+                       tile<8, 4>(), tile<5, 8>(), tile<6, 8>(),  tile<8, 8>(),  tile<9, 8>(),
+                       tile<10, 8>(), tile<12, 8>(), tile<14, 8>(), tile<16, 8>()};
+
+cudaError_t configure_kernel(const void* k) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+}
+
+cudaLaunchConfig_t launch_config(int grid, int cs, cudaStream_t s, cudaLaunchAttribute* at) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Clusters of `cs` CTAs the device can run at once (0 if it cannot run one).
+int max_clusters(int cs) {
+    cudaLaunchAttribute at[1];
+    const cudaLaunchConfig_t cfg = launch_config(cs * 16, cs, nullptr, at);
+    int n = 0;
+    for (const Tile& tl : kTiles) {
+        int m = 0;
+        if (cudaOccupancyMaxActiveClusters(&m, tl.kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        n = (tl.kernel == kTiles[0].kernel || m < n) ? m : n;
+    }
+    return n;
+}
+
+// Modelled cycles of one level of a CTA: the slabs' bytes at the L2-to-shared-memory
+// rate measured for one SM (~41 B/clk), against the scoring of 64 steps of 4
+// dimensions (per step the larger of 8 warps x (U + V) shared-memory loads and 2
+// warps per scheduler x U V FMAs; measured ~1.7x this), plus the fixed work of
+// reducing, exchanging and updating (~3 000 cycles).
+long long level_cycles(int cs, const Tile& tl) {
+    const long long stream = (long long)(kK / cs) * 1024 / 41;
+    const long long lds = 8 * (tl.U + tl.V), fma = 2 * tl.U * tl.V;
+    const long long score = 64 * (lds > fma ? lds : fma) * 17 / 10;
+    return (stream > score ? stream : score) + 3000;
+}
+
+}  // namespace
+
+cudaError_t encode_cluster_configure(Tables& t) {
+    t.cl_max8 = 0;
+    t.cl_max16 = 0;
+    for (const Tile& tl : kTiles)
+        if (configure_kernel(tl.kernel) != cudaSuccess) {
+            // no cluster form on this device: streaming steps take the other encoders
+            cudaGetLastError();
+            return cudaSuccess;
+        }
+    t.cl_max8 = max_clusters(8);
+    t.cl_max16 = max_clusters(16);
+    return cudaSuccess;
+}
+
+ClusterPlan plan_encode_cluster(const Tables& t, int B) {
+    ClusterPlan p{};
+    if (B <= 0) return p;
+    long long best = -1;
+    for (int cs = 8; cs <= 16; cs *= 2) {
+        const int nmax = cs == 8 ? t.cl_max8 : t.cl_max16;
+        if (nmax <= 0) continue;
+        const int fc = (B + nmax - 1) / nmax;
+        if (fc > kClusterMaxBlock) continue;
+        const int slice = kK / cs;
+        for (int i = 0; i < (int)(sizeof(kTiles) / sizeof(kTiles[0])); ++i) {
+            const Tile& tl = kTiles[i];
+            const int wc = slice / (8 * tl.V);
+            if (wc < 1 || 8 % wc != 0) continue;
+            const int rows = (8 / wc) * tl.U;
+            if (rows < fc || rows > kClusterMaxBlock) continue;
+            const long long c = level_cycles(cs, tl);
+            if (best < 0 || c < best) {
+                best = c;
+                p.cs = cs;
+                p.fc = fc;
+                p.nc = (B + fc - 1) / fc;
+                p.tile = i;
+                p.U = tl.U;
+                p.V = tl.V;
+            }
+        }
+    }
+    p.ok = best >= 0;
+    return p;
+}
+
+cudaError_t launch_encode_cluster(const Tables& t, const ClusterPlan& p, const void* z, int dtype,
+                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s) {
+    if (!p.ok) return cudaErrorInvalidValue;
+    ClusterArgs a;
+    a.C32 = t.C32;
+    a.Win32 = t.Win32;
+    a.cnorm = t.cnorm;
+    a.err = t.err;
+    a.stats = t.stats;
+    a.z = z;
+    a.dtype = dtype;
+    a.B = B;
+    a.n_q = n_q;
+    a.variant = variant;
+    a.cs = p.cs;
+    a.fc = p.fc;
+    a.codes = codes;
+    cudaLaunchAttribute at[1];
+    const cudaLaunchConfig_t cfg = launch_config(p.nc * p.cs, p.cs, s, at);
+    const CUtensorMap* tm = p.cs == 8 ? &t.tm_C32_8 : &t.tm_C32_16;
+    void* args[] = {const_cast<CUtensorMap*>(tm), &a};
+    return cudaLaunchKernelExC(&cfg, kTiles[p.tile].kernel, args);
+}
+
+}  // namespace mimi

@@ -43,8 +43,15 @@ constexpr int kSliceListFloats = 10;  // per row: 8 candidate keys, best, evicte
 // the sliced encoder 207-209 us from 256 to 511 frames, 215 us at 1024.
 constexpr int kSlicedMinFrames = 257;
 
+// Cluster form of the latency encoder (streaming steps): blocks of at most
+// kClusterMaxBlock frames, one per cluster of 8 or 16 CTAs, all clusters resident
+// at once (so steps of at most kClusterMaxBlock x the clusters the device runs).
+constexpr int kClusterMaxBlock = 32;
+
 struct Tables {
     int num_sms = 148;            // SMs of the handle's device (grid sizes)
+    int cl_max8 = 0;              // cluster form: clusters of 8 CTAs the device runs at once
+    int cl_max16 = 0;             //   and of 16 (0: that size is not available)
     // float32 originals
     float* C32 = nullptr;         // [Q][K][D] codebooks (0 semantic)
     float* Win32 = nullptr;       // [D][Din] W_in
@@ -71,6 +78,9 @@ struct Tables {
     CUtensorMap tm_C;             // Cbf as [Q*K rows][D cols]
     CUtensorMap tm_Whi;           // Win_hi as [D rows][Din cols]
     CUtensorMap tm_Wlo;           // Win_lo
+    CUtensorMap tm_C32_8;         // C32 as [Q*K rows][D cols] fp32, boxes of 32 columns x K / 8
+                                  // rows (the cluster form's slabs), 128-byte swizzle
+    CUtensorMap tm_C32_16;        // the same with K / 16 rows
 };
 
 // prep.cu
@@ -114,6 +124,22 @@ cudaError_t encode_wide_configure();  // once per device, before the first launc
 cudaError_t launch_encode_wide(const Tables& t, const WidePlan& p, const void* z, int dtype, int B,
                                int n_q, int variant, int16_t* codes, cudaStream_t s,
                                bool rescan_list = false);
+// encode_cluster.cu
+struct ClusterPlan {
+    bool ok = false;  // false: no cluster form, or more than kClusterMaxBlock frames per cluster
+    int cs = 0;       // CTAs per cluster (8 or 16)
+    int nc = 0;       // clusters (one frame block each)
+    int fc = 0;       // frames per cluster (the last may have fewer)
+    int tile = 0;     // thread tile (index of the built tiles)
+    int U = 0, V = 0; //   U frames x V codewords per lane quad
+};
+// once per handle, after encode_wide_configure: sets t.cl_max8 and t.cl_max16 (0
+// for a cluster size the device cannot run; not an error)
+cudaError_t encode_cluster_configure(Tables& t);
+ClusterPlan plan_encode_cluster(const Tables& t, int B);
+// Reads only the tables: launches on several streams may overlap.
+cudaError_t launch_encode_cluster(const Tables& t, const ClusterPlan& p, const void* z, int dtype,
+                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s);
 // selftest.cu: a kernel whose wait can never complete (which 0: an mbarrier,
 // as the tensor-core encoder waits; 1: a group barrier, as the wide encoder
 // waits); it times out after ~50 ms and records MIMI_DEV_ERR_TIMEOUT.
