@@ -63,17 +63,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x 256 rows
 // (32 KiB: one stage of the tensor-core encoder's ring), 128-byte swizzle: the
 // layout the UMMA shared-memory descriptors expect.
-// 2-D fp32 tensor [rows][cols] (row-major), boxes of 32 columns x box_rows rows
-// (one 128-byte row per codeword), 128-byte swizzle: the cluster encoder's slabs.
-bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                   uint32_t box_rows) {
+// fp32 tensor [rows][256] (row-major) seen as slabs: dimension 0 the 32 columns of
+// a slab, 1 the rows (1024-byte stride), 2 the 8 slabs of a row (128-byte stride);
+// boxes of 32 columns x box_rows rows x box_slabs slabs (64 KiB), 128-byte swizzle:
+// the cluster encoder's stages, each slab's rows contiguous in shared memory.
+bool make_tmap_slabs(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 4};
-    const cuuint32_t box[2] = {32, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+    const cuuint64_t dims[3] = {32, rows, 8};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 4, 128};
+    const cuuint32_t box[3] = {32, box_rows, 65536 / (box_rows * 128)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -218,8 +219,8 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
         return MIMI_RVQ_ECUDA;
     }
     // the cluster form needs its slab maps; a size without one stays off
-    if (!make_tmap_f32(&t.tm_C32_8, t.C32, (uint64_t)kQ * kK, kD, kK / 8)) t.cl_max8 = 0;
-    if (!make_tmap_f32(&t.tm_C32_16, t.C32, (uint64_t)kQ * kK, kD, kK / 16)) t.cl_max16 = 0;
+    if (!make_tmap_slabs(&t.tm_C32_8, t.C32, (uint64_t)kQ * kK, kK / 8)) t.cl_max8 = 0;
+    if (!make_tmap_slabs(&t.tm_C32_16, t.C32, (uint64_t)kQ * kK, kK / 16)) t.cl_max16 = 0;
     *out = h;
     return MIMI_RVQ_OK;
 }

@@ -47,9 +47,8 @@ using lat::umin64;
 
 constexpr int kSlabDims = 32;                        // dimensions per slab (128 bytes per codeword)
 constexpr int kSlabsPerLevel = kD / kSlabDims;       // 8
-constexpr int NST = 4;                               // slab stages
-constexpr int kMaxSlice = kK / 8;                    // codewords per CTA in clusters of 8
-constexpr int STAGE_BYTES = kMaxSlice * 128;         // 32 KiB
+constexpr int NST = 2;                               // stages
+constexpr int STAGE_BYTES = 64 * 1024;               // a stage: 64 KiB of slabs (2 or 4)
 constexpr int YSTRIDE = 32;                          // row stride (floats) of the projection block
 constexpr int R_OFF = NST * STAGE_BYTES;             // bytes: r rows
 constexpr int Y_OFF = R_OFF + kClusterMaxBlock * RSTRIDE * 4;      // projection block
@@ -104,15 +103,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wf = wid / WC, wc = wid % WC;
     const int k_base = rank * slice;
     const int DO = kD / cs;             // projection outputs of this CTA: [rank * DO, rank * DO + DO)
-    const int total = a.n_q * kSlabsPerLevel;
-    const uint32_t stage_tx = (uint32_t)slice * 128u;
+    const int slab_bytes = slice * 128;
+    const int nb = STAGE_BYTES / slab_bytes;   // slabs per stage: 2 (clusters of 8) or 4 (of 16)
+    const int spl = kSlabsPerLevel / nb;       // stages per level
+    const int total = a.n_q * spl;
 
-    // slab s: dimensions [32 (s % 8), + 32) of this CTA's codewords of level s / 8
-    auto issue = [&](int s) {
-        uint64_t* bar = &full[s % NST];
-        mbar_arrive_expect_tx(bar, stage_tx);
-        tma_load_2d(sm + (s % NST) * STAGE_BYTES, &tm_C32, bar, (s % kSlabsPerLevel) * kSlabDims,
-                    (s / kSlabsPerLevel) * kK + k_base);
+    // stage t: slabs [nb (t % spl), + nb) of this CTA's codewords of level t / spl, one
+    // box (the slab index is the map's outer dimension)
+    auto issue = [&](int t) {
+        uint64_t* bar = &full[t % NST];
+        mbar_arrive_expect_tx(bar, (uint32_t)STAGE_BYTES);
+        tma_load_3d(sm + (t % NST) * STAGE_BYTES, &tm_C32, bar, 0, (t / spl) * kK + k_base,
+                    (t % spl) * nb);
     };
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this lane's codewords (row within the CTA's slice: cw0 + 8v) and frames (fr0 + u)
     const int cw0 = wc * 8 * V + g;
     const int fr0 = wf * U;
-    int s = 0;  // slab index over all levels
+    int s = 0;  // stage index over all levels
     for (int l = 0; l < a.n_q; ++l) {
         // minima by level parity: a slot is rewritten two levels later, after the
         // barrier that every CTA reaches only once it has read it
@@ -208,24 +210,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < U; ++u)
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
-        for (int j = 0; j < kSlabsPerLevel; ++j, ++s) {
+        for (int tt = 0; tt < spl; ++tt, ++s) {
             mbar_wait(&full[s % NST], (uint32_t)(s / NST) & 1u, abort, a.err);
-            // codeword row cw0 + 8v of the stage: 128 bytes, 16-byte unit x at x ^ (row & 7),
-            // and row & 7 = g
-            const uint8_t* cb = sm + (s % NST) * STAGE_BYTES + cw0 * 128 + 4 * w;
-            const float* rb = r_s + fr0 * RSTRIDE + j * kSlabDims + w;
+#pragma unroll 1
+            for (int jj = 0; jj < nb; ++jj) {
+                // codeword row cw0 + 8v of slab jj: 128 bytes, 16-byte unit x at x ^ (row & 7),
+                // and row & 7 = g
+                const uint8_t* cb = sm + (s % NST) * STAGE_BYTES + jj * slab_bytes + cw0 * 128 + 4 * w;
+                const float* rb = r_s + fr0 * RSTRIDE + (tt * nb + jj) * kSlabDims + w;
 #pragma unroll
-            for (int i = 0; i < kSlabDims; i += 4) {
-                const int off = ((i >> 2) ^ g) << 4;
-                float cv[V], rv[U];
+                for (int i = 0; i < kSlabDims; i += 4) {
+                    const int off = ((i >> 2) ^ g) << 4;
+                    float cv[V], rv[U];
 #pragma unroll
-                for (int v = 0; v < V; ++v) cv[v] = *reinterpret_cast<const float*>(cb + v * 1024 + off);
+                    for (int v = 0; v < V; ++v) cv[v] = *reinterpret_cast<const float*>(cb + v * 1024 + off);
 #pragma unroll
-                for (int u = 0; u < U; ++u) rv[u] = rb[u * RSTRIDE + i];
+                    for (int u = 0; u < U; ++u) rv[u] = rb[u * RSTRIDE + i];
 #pragma unroll
-                for (int u = 0; u < U; ++u)
+                    for (int u = 0; u < U; ++u)
 #pragma unroll
-                    for (int v = 0; v < V; ++v) acc[u][v] = fmaf(rv[u], cv[v], acc[u][v]);
+                        for (int v = 0; v < V; ++v) acc[u][v] = fmaf(rv[u], cv[v], acc[u][v]);
+                }
             }
             __syncthreads();  // every warp is done with the stage
             if (tid == 0 && s + NST < total) issue(s + NST);
