@@ -38,7 +38,6 @@
 namespace mimi {
 namespace {
 
-using lat::kProjItems;
 using lat::kThreads;
 using lat::load_latent4;
 using lat::pack_key;
@@ -63,6 +62,42 @@ static_assert(BAR_OFF % 8 == 0 && MK_OFF % 8 == 0 && RED_OFF % 8 == 0, "alignmen
 // the projection stages F + kD / CS rows of all kDin + 1 columns over the slab stages and the
 // r rows, before either is in use
 static_assert((kClusterMaxBlock + kD / 8) * (kDin + 1) * 4 <= Y_OFF, "projection staging fits");
+
+// y = W_in . z for a tile of PF frames (rows pf.., clamped to F - 1: computed,
+// never stored) x PD outputs (rows pd..) of the staged latents and W_in rows (row
+// stride kDin + 1): every output a sequential FMA chain over all kDin columns (the
+// full scan's order), each staged value read once for the tile's chains.
+template <int PF, int PD>
+__device__ __forceinline__ void proj_tile(const float* z_s, const float* w_s, int pf, int pd, int F,
+                                          float* y_s) {
+    constexpr int JS = kDin + 1;
+    float acc[PF][PD];
+#pragma unroll
+    for (int i = 0; i < PF; ++i)
+#pragma unroll
+        for (int k = 0; k < PD; ++k) acc[i][k] = 0.f;
+    const float* zr[PF];
+#pragma unroll
+    for (int i = 0; i < PF; ++i) zr[i] = z_s + min(pf + i, F - 1) * JS;
+    const float* wr = w_s + pd * JS;
+#pragma unroll 8
+    for (int j = 0; j < kDin; ++j) {
+        float zv[PF], wv[PD];
+#pragma unroll
+        for (int i = 0; i < PF; ++i) zv[i] = zr[i][j];
+#pragma unroll
+        for (int k = 0; k < PD; ++k) wv[k] = wr[k * JS + j];
+#pragma unroll
+        for (int i = 0; i < PF; ++i)
+#pragma unroll
+            for (int k = 0; k < PD; ++k) acc[i][k] = fmaf(wv[k], zv[i], acc[i][k]);
+    }
+#pragma unroll
+    for (int i = 0; i < PF; ++i)
+        if (pf + i < F)
+#pragma unroll
+            for (int k = 0; k < PD; ++k) y_s[(pf + i) * YSTRIDE + pd + k] = acc[i][k];
+}
 
 struct ClusterArgs {
     const float* C32;
@@ -125,25 +160,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- y = W_in . z for the cluster's F frames x this CTA's DO outputs, each a
     //      sequential FMA chain over j (the full scan's order); latents and W_in rows
-    //      staged whole (every load in flight at once) over the slab stages and r rows
+    //      staged whole (every load in flight at once) over the slab stages and r rows.
+    //      Shared-memory reads bound the chains, so for more than six frames a
+    //      thread keeps 2 or 4 frames x 2 outputs in registers and each value it
+    //      reads feeds several chains; for a few frames, one chain per thread.
     {
         const int d0 = rank * DO;
-        const int items = F * DO;
         constexpr int JC = kDin, JS = JC + 1, J4 = JC / 4;
         float* z_s = reinterpret_cast<float*>(sm);   // [F][JS]
         float* w_s = z_s + F * JS;                   // [DO][JS]
-        const int nq_items = (items + kThreads - 1) / kThreads;  // uniform over the CTA
-        int zo[kProjItems], wo[kProjItems];
-        float acc[kProjItems];
-#pragma unroll
-        for (int q = 0; q < kProjItems; ++q) {
-            const int it = tid + q * kThreads;
-            const bool act = it < items;
-            zo[q] = act ? (it / DO) * JS : 0;
-            wo[q] = act ? (it % DO) * JS : 0;
-            acc[q] = 0.f;
-        }
-        for (int j0 = 0; j0 < kDin; j0 += JC) {
+        {
+            const int j0 = 0;
             __syncthreads();
             const int nz = F * J4, nt = (F + DO) * J4;
             for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
@@ -170,12 +197,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncthreads();
-            lat::proj_chain_any(nq_items, z_s, w_s, zo, wo, acc, JC);
-        }
-#pragma unroll
-        for (int q = 0; q < kProjItems; ++q) {
-            const int it = tid + q * kThreads;
-            if (it < items) y_s[(it / DO) * YSTRIDE + it % DO] = acc[q];
+            const int pf_n = F <= 6 ? 1 : F <= 12 ? 2 : 4, pd_n = F <= 6 ? 1 : 2;
+            const int nob = DO / pd_n, nfb = (F + pf_n - 1) / pf_n;
+            if (tid < nfb * nob) {
+                const int pf = (tid / nob) * pf_n, pd = (tid % nob) * pd_n;
+                if (pf_n == 1) proj_tile<1, 1>(z_s, w_s, pf, pd, F, y_s);
+                else if (pf_n == 2) proj_tile<2, 2>(z_s, w_s, pf, pd, F, y_s);
+                else proj_tile<4, 2>(z_s, w_s, pf, pd, F, y_s);
+            }
         }
     }
     __syncthreads();  // the staging is read: the stages take the first slabs
