@@ -164,15 +164,17 @@ def test_streaming_step(batch):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_small_streaming_steps_equal_the_full_scan(dtype):
-    """Steps of at most 256 frames run the latency encoder, whose scores are the float32 full
-    scan's (same sums in the same order): every code equals encode_scan's, near ties
-    included. Sizes span one to four frame groups, ragged group tails and every thread-tile
-    shape."""
+    """Steps of at most 480 frames run the float32 latency encoder on thread-block clusters,
+    whose scores are the full scan's (same sums in the same order): every code equals
+    encode_scan's, near ties included. Sizes span clusters of 16 and of 8 CTAs, one to 32
+    frames per cluster with ragged last clusters, every thread tile and every projection
+    tile."""
     model, frames = synth.streaming_step(1024, calls=1)
     q = quantizer(model)
     z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
     zd = to_device(np.ascontiguousarray(z))
-    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 200, 255, 256)
+    sizes = (1, 2, 3, 15, 16, 17, 33, 45, 63, 64, 65, 90, 100, 127, 128, 129, 180, 200, 255,
+             256, 257, 300, 361, 384, 450, 479, 480)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         scan = q.encode_scan(zd[:b]).cpu().numpy()
@@ -184,7 +186,7 @@ def test_small_streaming_steps_equal_the_full_scan(dtype):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_sliced_streaming_steps_match_the_oracle(dtype):
-    """Steps of more than 256 frames run the codebook-sliced tensor-core encoder (8 CTAs per
+    """Steps of more than 480 frames run the codebook-sliced tensor-core encoder (8 CTAs per
     128-frame group, candidate lists exchanged through global memory): codes equal the
     oracle's outside near-ties and the batch tensor-core encoder's on every other frame,
     for full and ragged groups, up to the 18 groups that fit the device at once."""
@@ -195,7 +197,7 @@ def test_sliced_streaming_steps_match_the_oracle(dtype):
     ref, db, ds = oracle.encode(z, model.W_in, model.C)
     near = oracle.near_tie(db, ds)
     enc0, _ = q.stats()
-    sizes = (257, 300, 384, 511, 512, 513, 700, 896, 1000, 1024, 2304)
+    sizes = (481, 511, 512, 513, 700, 896, 1000, 1024, 2304)
     for b in sizes:
         step = q.encode_step(zd[:b]).cpu().numpy()
         assert_codes_match(step, ref[:b], db[:b], ds[:b], f"sliced step B={b}")
@@ -235,13 +237,35 @@ def test_streaming_step_fewer_codebooks_and_variant():
     model, frames = synth.streaming_step(600, calls=1)
     q = quantizer(model)
     zd = to_device(np.ascontiguousarray(frames[0]))
-    for b in (100, 600):   # latency encoder, sliced tensor-core encoder
+    for b in (100, 600):   # cluster latency encoder, sliced tensor-core encoder
         for n_q, variant in ((1, 0), (5, 0), (8, 1), (3, 1)):
             step = q.encode_step(zd[:b], n_q=n_q, variant=variant).cpu().numpy()
             assert step.shape == (b, n_q)
             ref, db, ds = oracle.encode(frames[0][:b], model.W_in, model.C, n_q=n_q,
                                         variant=variant)
             assert_codes_match(step, ref, db, ds, f"step B={b} n_q={n_q} variant={variant}")
+    assert q.get_error() == 0
+
+
+def test_cluster_steps_on_two_streams_at_once():
+    """The cluster form reads only the handle's tables, so steps launched on two streams with
+    no ordering between them may overlap: both return the full scan's codes."""
+    model, frames = synth.streaming_step(192, calls=2)
+    q = quantizer(model)
+    za = to_device(np.ascontiguousarray(frames[0][:128]))
+    zb = to_device(np.ascontiguousarray(frames[1][:64]))
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    oa = torch.empty((128, 8), dtype=torch.int16, device="cuda")
+    ob = torch.empty((64, 8), dtype=torch.int16, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(20):
+        with torch.cuda.stream(sa):
+            q.encode_step(za, out=oa, stream=sa)
+        with torch.cuda.stream(sb):
+            q.encode_step(zb, out=ob, stream=sb)
+    torch.cuda.synchronize()
+    assert np.array_equal(oa.cpu().numpy(), q.encode_scan(za).cpu().numpy())
+    assert np.array_equal(ob.cpu().numpy(), q.encode_scan(zb).cpu().numpy())
     assert q.get_error() == 0
 
 
@@ -260,9 +284,9 @@ def test_streaming_step_large_batch(batch):
 
 @pytest.mark.parametrize("batch", [1, 128, 1024])
 def test_streaming_step_in_a_cuda_graph(batch):
-    """The group barriers of both streaming encoders return to their starting state after
-    every launch, so a captured step replays correctly on new inputs (the same codes as an
-    uncaptured step)."""
+    """A captured step replays correctly on new inputs (the same codes as an uncaptured step):
+    the cluster form keeps no state between launches, and the sliced form's group barriers
+    return to their starting state after every launch."""
     model, frames = synth.streaming_step(batch, calls=4)
     q = quantizer(model)
     static_in = to_device(np.ascontiguousarray(frames[0]))
