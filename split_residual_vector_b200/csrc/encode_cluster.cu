@@ -231,9 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // minima by level parity: a slot is rewritten two levels later, after the
         // barrier that every CTA reaches only once it has read it
         unsigned long long* mk = mk_s + (l & 1) * kClusterMaxBlock;
-        float cnv[V];
+        // after the level's scores this lane holds the dots of codewords vq + k, k < V / 4
+        // (see below): their ||c||^2 now, so the loads overlap the scoring
+        const int vq = (w & 1) * (V / 2) + (w >> 1) * (V / 4);
+        float cnv[V / 4];
 #pragma unroll
-        for (int v = 0; v < V; ++v) cnv[v] = __ldg(a.cnorm + (size_t)l * kK + k_base + cw0 + 8 * v);
+        for (int k = 0; k < V / 4; ++k)
+            cnv[k] = __ldg(a.cnorm + (size_t)l * kK + k_base + cw0 + 8 * (vq + k));
         float acc[U][V];
 #pragma unroll
         for (int u = 0; u < U; ++u)
@@ -264,20 +268,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();  // every warp is done with the stage
             if (tid == 0 && s + NST < total) issue(s + NST);
         }
-        // dot = (p0 + p1) + (p2 + p3) across the quad, then the minimum key per frame over
-        // the warp's codewords and one shared atomic per warp and frame
+        // dot = (p0 + p1) + (p2 + p3) across the quad as a reduce-scatter: lanes w and
+        // w ^ 1 add their partials of the codeword half each keeps (w & 1 picks it), then
+        // lanes w and w ^ 2 those of the quarter each keeps (w & 2), so lane w ends with
+        // the dots of codewords vq + k, k < V / 4 (3 UV / 4 shuffles instead of 2 UV; the
+        // sums are the same, each addition being commutative). Then the minimum key per
+        // frame over the warp and one slot per warp and frame.
 #pragma unroll
         for (int u = 0; u < U; ++u) {
+            float h[V / 2];
+#pragma unroll
+            for (int k = 0; k < V / 2; ++k) {
+                const float lo = acc[u][k], hi = acc[u][k + V / 2];
+                const float send = (w & 1) ? lo : hi, keep = (w & 1) ? hi : lo;
+                h[k] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            }
             unsigned long long best = ~0ull;
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                float p = acc[u][v];
-                p = p + __shfl_xor_sync(0xffffffffu, p, 1);
-                p = p + __shfl_xor_sync(0xffffffffu, p, 2);
-                best = umin64(best, pack_key(fmaf(-2.f, p, cnv[v]), k_base + cw0 + 8 * v));
+            for (int k = 0; k < V / 4; ++k) {
+                const float a0 = h[k], a1 = h[k + V / 4];
+                const float send = (w & 2) ? a0 : a1, keep = (w & 2) ? a1 : a0;
+                const float dot = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                best = umin64(best, pack_key(fmaf(-2.f, dot, cnv[k]), k_base + cw0 + 8 * (vq + k)));
             }
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) best = umin64(best, __shfl_xor_sync(0xffffffffu, best, o));
+            for (int o = 1; o < 32; o <<= 1) best = umin64(best, __shfl_xor_sync(0xffffffffu, best, o));
             if (lane == 0) red_s[wid * 16 + u] = best;
         }
         __syncthreads();
