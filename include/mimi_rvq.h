@@ -100,14 +100,18 @@ int mimi_rvq_encode(mimi_rvq_t h, const void *latents, int dtype, int64_t N,
 /*
  * Streaming step: one 512-d frame for each of B concurrent streams (B >= 0),
  * frames [B][512] -> codes [B][8]. The quantiser keeps no state between
- * frames, so a step is an encode of B frames tuned for latency: up to 256
- * frames run a float32 kernel spread over every SM (its codes equal
- * mimi_rvq_encode_scan's); 257 to 2304 frames (while 8 CTAs per 128-frame
- * group fit the device) run a codebook-sliced form of the tensor-core encoder
- * (one launch; codes as the batch encoder's); larger steps run the batch
- * encoder. Allocates nothing, never synchronises the host, and may be captured
- * in a CUDA graph. Steps on one handle share its scratch: issue them in stream
- * order.
+ * frames, so a step is an encode of B frames tuned for latency: up to 32
+ * frames per thread-block cluster the device runs at once (480 on B200:
+ * 15 clusters of 8 CTAs) run a float32 kernel on clusters that split the
+ * codebooks (its codes equal mimi_rvq_encode_scan's; it keeps no state, so
+ * such steps may run on several streams at once); larger steps up to 2304
+ * frames (while 8 CTAs per 128-frame group fit the device) run a
+ * codebook-sliced form of the tensor-core encoder (one launch; codes as the
+ * batch encoder's); larger steps run the batch encoder. On a device without
+ * clusters, steps of up to 256 frames run a float32 kernel over groups of CTAs
+ * (also the full scan's codes). Allocates nothing, never synchronises the
+ * host, and may be captured in a CUDA graph. Steps other than the cluster
+ * form share the handle's scratch: issue them in stream order.
  */
 int mimi_rvq_encode_step(mimi_rvq_t h, const void *frames, int dtype, int B,
                          int16_t *codes, struct CUstream_st *stream);

@@ -1,4 +1,6 @@
-// encode_wide.cu -- latency encode for small batches (the streaming step).
+// encode_wide.cu -- latency encode for small batches, group form: the float32
+// re-encode of the frames the batch tensor-core encoder could not certify, and
+// streaming steps on a device without the cluster form (encode_cluster.cu).
 //
 // The tensor-core encoder gives each 128-frame tile to one SM, which then
 // walks the 8 codebooks in series: a batch of a few frames occupies one SM and
@@ -18,8 +20,7 @@
 // split over the group's CTAs as frame blocks x output blocks and exchanged
 // through global memory behind one more barrier. Every sum is taken in the
 // float32 full scan's order, so the codes are the ones mimi_rvq_encode_scan
-// returns. It serves streaming steps of up to 256 frames and the re-encode of
-// the frames the batch tensor-core encoder could not certify.
+// returns.
 //
 // Codeword chunks are double-buffered with cp.async; the next level's first
 // chunk does not depend on the winners, so its copy overlaps the barrier.

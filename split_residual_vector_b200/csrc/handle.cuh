@@ -19,9 +19,10 @@ constexpr int kQ = 8;         // codebooks: 0 semantic, 1..7 acoustic
 // list cannot overflow).
 constexpr int64_t kRescanCapacity = 1 << 20;
 
-// Largest batch the latency (wide) encoder takes: streaming steps up to
-// kSlicedMinFrames - 1 frames, and the float32 re-encode of the frames the batch
-// tensor-core encoder could not certify, 1024 at a time.
+// Largest batch the group form of the latency encoder takes: the float32
+// re-encode of the frames the batch tensor-core encoder could not certify, 1024
+// at a time, and (on a device without the cluster form) streaming steps up to
+// kSlicedMinFrames - 1 frames.
 constexpr int kWideMaxFrames = 1024;
 constexpr int kWideGroupFrames = 64;  // frames per group of the latency encoder
 constexpr int kWideMaxGroups = 64;    // group barriers (the last one is the wait self-test's)
@@ -36,11 +37,12 @@ constexpr int kSlices = 8;
 constexpr int kSliceMaxGroups = 18;   // 18 x 8 CTAs fit on 148 SMs, one CTA each
 constexpr int kSliceBarBase = 32;
 constexpr int kSliceListFloats = 10;  // per row: 8 candidate keys, best, evicted
-// Streaming steps of at least this many frames take the sliced tensor-core
-// encoder (when its CTAs fit the device); smaller ones the float32 latency encoder.
-// Measured per step on B200: the latency encoder 52 us at 1 frame, 105 us at 128,
-// 136 us at 256, but 211-219 us from 320 to 511 frames (five groups and more);
-// the sliced encoder 207-209 us from 256 to 511 frames, 215 us at 1024.
+// Streaming steps the cluster form cannot take (more than 32 frames per cluster)
+// run the sliced tensor-core encoder when its CTAs fit the device. On a device
+// without the cluster form, steps of fewer than kSlicedMinFrames frames run the
+// group form of the latency encoder instead. Measured per step on B200: the group
+// form 52 us at 1 frame, 105 us at 128, 136 us at 256, 211-219 us from 320 to 511
+// frames; the sliced encoder 207-209 us from 256 to 511 frames, 215 us at 1024.
 constexpr int kSlicedMinFrames = 257;
 
 // Cluster form of the latency encoder (streaming steps): blocks of at most
