@@ -31,8 +31,9 @@
 // banks (a warp's 8 quads take 8 consecutive codewords); the partials are
 // combined at the end of the level by two shuffles, (p0 + p1) + (p2 + p3),
 // the scan's order. The CTA's codewords arrive by TMA as slabs of 32
-// dimensions (one 128-byte row per codeword, 128-byte swizzle) through a
-// 4-stage ring; one thread refills a stage once every warp is done with it.
+// dimensions (one 128-byte row per codeword, 128-byte swizzle) in two 64 KiB
+// stages, each filled by one 3-D box of 2 or 4 slabs; one thread refills a
+// stage once every warp is done with it.
 #include "latency_common.cuh"
 
 namespace mimi {
@@ -166,45 +167,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      reads feeds several chains; for a few frames, one chain per thread.
     {
         const int d0 = rank * DO;
-        constexpr int JC = kDin, JS = JC + 1, J4 = JC / 4;
+        constexpr int JS = kDin + 1, J4 = kDin / 4;
         float* z_s = reinterpret_cast<float*>(sm);   // [F][JS]
         float* w_s = z_s + F * JS;                   // [DO][JS]
-        {
-            const int j0 = 0;
-            __syncthreads();
-            const int nz = F * J4, nt = (F + DO) * J4;
-            for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
-                float4 v[16];
+        const int nz = F * J4, nt = (F + DO) * J4;
+        for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
+            float4 v[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * kThreads;
-                    if (e < nz)
-                        v[u] = load_latent4(a.z, a.dtype, (int64_t)(f0 + e / J4) * kDin + j0 + 4 * (e % J4));
-                    else if (e < nt)
-                        v[u] = __ldg(reinterpret_cast<const float4*>(
-                            a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + j0 + 4 * ((e - nz) % J4)));
-                }
+            for (int u = 0; u < 16; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < nz)
+                    v[u] = load_latent4(a.z, a.dtype, (int64_t)(f0 + e / J4) * kDin + 4 * (e % J4));
+                else if (e < nt)
+                    v[u] = __ldg(reinterpret_cast<const float4*>(
+                        a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + 4 * ((e - nz) % J4)));
+            }
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * kThreads;
-                    if (e < nt) {
-                        float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
-                        d[0] = v[u].x;
-                        d[1] = v[u].y;
-                        d[2] = v[u].z;
-                        d[3] = v[u].w;
-                    }
+            for (int u = 0; u < 16; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < nt) {
+                    float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
+                    d[0] = v[u].x;
+                    d[1] = v[u].y;
+                    d[2] = v[u].z;
+                    d[3] = v[u].w;
                 }
             }
-            __syncthreads();
-            const int pf_n = F <= 6 ? 1 : F <= 12 ? 2 : 4, pd_n = F <= 6 ? 1 : 2;
-            const int nob = DO / pd_n, nfb = (F + pf_n - 1) / pf_n;
-            if (tid < nfb * nob) {
-                const int pf = (tid / nob) * pf_n, pd = (tid % nob) * pd_n;
-                if (pf_n == 1) proj_tile<1, 1>(z_s, w_s, pf, pd, F, y_s);
-                else if (pf_n == 2) proj_tile<2, 2>(z_s, w_s, pf, pd, F, y_s);
-                else proj_tile<4, 2>(z_s, w_s, pf, pd, F, y_s);
-            }
+        }
+        __syncthreads();
+        const int pf_n = F <= 6 ? 1 : F <= 12 ? 2 : 4, pd_n = F <= 6 ? 1 : 2;
+        const int nob = DO / pd_n, nfb = (F + pf_n - 1) / pf_n;
+        if (tid < nfb * nob) {
+            const int pf = (tid / nob) * pf_n, pd = (tid % nob) * pd_n;
+            if (pf_n == 1) proj_tile<1, 1>(z_s, w_s, pf, pd, F, y_s);
+            else if (pf_n == 2) proj_tile<2, 2>(z_s, w_s, pf, pd, F, y_s);
+            else proj_tile<4, 2>(z_s, w_s, pf, pd, F, y_s);
         }
     }
     __syncthreads();  // the staging is read: the stages take the first slabs
