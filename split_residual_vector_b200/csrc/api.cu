@@ -111,6 +111,14 @@ cudaError_t dalloc(T** p, size_t count) {
 // with the float32 wide encoder, 1024 at a time (16 groups of 64 share the GPU).
 cudaError_t rescan(mimi_rvq_t h, const void* z, int dtype, int n_q, int variant, int16_t* codes,
                    cudaStream_t s) {
+    // the cluster form, 32 frames per cluster per pass, where the device runs it
+    const int per_pass = mimi::kClusterMaxBlock * h->t.cl_max8;
+    if (per_pass > 0) {
+        const mimi::ClusterPlan cp = mimi::plan_encode_cluster(h->t, per_pass);
+        if (cp.ok && cp.cs == 8 && cp.U == 16 && cp.V == 8)  // the list mode's tile
+            return mimi::launch_encode_cluster(h->t, cp, z, dtype, per_pass, n_q, variant, codes, s,
+                                               true);
+    }
     const int batch = mimi::kWideMaxFrames;
     const mimi::WidePlan p = mimi::plan_encode_wide(batch, h->num_sms);
     if (!p.ok) return cudaErrorInvalidConfiguration;

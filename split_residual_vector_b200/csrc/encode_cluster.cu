@@ -57,7 +57,8 @@ constexpr int WIN_OFF = MK_OFF + 2 * kClusterMaxBlock * 8;         // [block] wi
 constexpr int BAR_OFF = WIN_OFF + kClusterMaxBlock * 4;            // [NST] slab barriers
 constexpr int ABORT_OFF = BAR_OFF + NST * 8;
 constexpr int RED_OFF = ABORT_OFF + 16;                            // [8 warps][16] per-warp minima
-constexpr int SMEM_BYTES = RED_OFF + 8 * 16 * 8 + 1024;  // + alignment of the swizzled stages
+constexpr int FRAME_OFF = RED_OFF + 8 * 16 * 8;                    // [block] frame indices
+constexpr int SMEM_BYTES = FRAME_OFF + kClusterMaxBlock * 4 + 1024;  // + alignment of the stages
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 static_assert(BAR_OFF % 8 == 0 && MK_OFF % 8 == 0 && RED_OFF % 8 == 0, "alignment");
 // the projection stages F + kD / CS rows of all kDin + 1 columns over the slab stages and the
@@ -111,11 +112,17 @@ struct ClusterArgs {
     int cs;   // CTAs per cluster
     int fc;   // frames per cluster (the last cluster may have fewer)
     int16_t* codes;
+    // list mode (re-encode of the frames the tensor-core encoder could not certify):
+    // frames list[0 .. min(*list_count, list_cap)), nc x fc per pass; nullptr: frames 0..B-1
+    const int* list;
+    const int* list_count;
+    int list_cap;
 };
 
 // Thread tile U frames x V codewords per lane quad; warps split as WF (frame
-// blocks of U) x WC (codeword blocks of 8V), WC = (K / CS) / (8V).
-template <int U, int V>
+// blocks of U) x WC (codeword blocks of 8V), WC = (K / CS) / (8V). kList: the
+// list mode (passes over the listed frames); otherwise one block of frames.
+template <int U, int V, bool kList>
 __global__ void __launch_bounds__(kThreads, 1)
     k_encode_cluster(const __grid_constant__ CUtensorMap tm_C32, ClusterArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -124,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* y_s = reinterpret_cast<float*>(sm + Y_OFF);
     unsigned long long* mk_s = reinterpret_cast<unsigned long long*>(sm + MK_OFF);
     int* win_s = reinterpret_cast<int*>(sm + WIN_OFF);
+    int* frame_s = reinterpret_cast<int*>(sm + FRAME_OFF);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + BAR_OFF);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + ABORT_OFF);
     unsigned long long* red_s = reinterpret_cast<unsigned long long*>(sm + RED_OFF);
@@ -132,8 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = lane >> 2, w = lane & 3;
     const int cs = a.cs;
     const int rank = (int)cluster_ctarank();
-    const int f0 = (blockIdx.x / cs) * a.fc;
-    const int F = min(a.fc, a.B - f0);  // >= 1: the plan launches no empty cluster
+    const int nc = gridDim.x / cs, cl = blockIdx.x / cs;
+    int n_frames = a.B;
+    if constexpr (kList) {
+        n_frames = min(__ldcg(a.list_count), a.list_cap);
+        if (blockIdx.x == 0 && tid == 0 && n_frames > 0)
+            atomicAdd(&a.stats[1], (unsigned long long)n_frames);
+    }
     const int slice = kK / cs;
     const int WC = slice / (8 * V);
     const int wf = wid / WC, wc = wid % WC;
@@ -144,12 +157,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int spl = kSlabsPerLevel / nb;       // stages per level
     const int total = a.n_q * spl;
 
-    // stage t: slabs [nb (t % spl), + nb) of this CTA's codewords of level t / spl, one
-    // box (the slab index is the map's outer dimension)
-    auto issue = [&](int t) {
-        uint64_t* bar = &full[t % NST];
+    // stage t of a pass (sg of the launch): slabs [nb (t % spl), + nb) of this CTA's
+    // codewords of level t / spl, one box (the slab index is the map's outer dimension)
+    auto issue = [&](int sg, int t) {
+        uint64_t* bar = &full[sg % NST];
         mbar_arrive_expect_tx(bar, (uint32_t)STAGE_BYTES);
-        tma_load_3d(sm + (t % NST) * STAGE_BYTES, &tm_C32, bar, 0, (t / spl) * kK + k_base,
+        tma_load_3d(sm + (sg % NST) * STAGE_BYTES, &tm_C32, bar, 0, (t / spl) * kK + k_base,
                     (t % spl) * nb);
     };
     if (tid == 0) {
@@ -159,192 +172,213 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // ---- y = W_in . z for the cluster's F frames x this CTA's DO outputs, each a
-    //      sequential FMA chain over j (the full scan's order); latents and W_in rows
-    //      staged whole (every load in flight at once) over the slab stages and r rows.
-    //      Shared-memory reads bound the chains, so for more than six frames a
-    //      thread keeps 2 or 4 frames x 2 outputs in registers and each value it
-    //      reads feeds several chains; for a few frames, one chain per thread.
-    {
-        const int d0 = rank * DO;
-        constexpr int JS = kDin + 1, J4 = kDin / 4;
-        float* z_s = reinterpret_cast<float*>(sm);   // [F][JS]
-        float* w_s = z_s + F * JS;                   // [DO][JS]
-        const int nz = F * J4, nt = (F + DO) * J4;
-        for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
-            float4 v[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int e = e0 + u * kThreads;
-                if (e < nz)
-                    v[u] = load_latent4(a.z, a.dtype, (int64_t)(f0 + e / J4) * kDin + 4 * (e % J4));
-                else if (e < nt)
-                    v[u] = __ldg(reinterpret_cast<const float4*>(
-                        a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + 4 * ((e - nz) % J4)));
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int e = e0 + u * kThreads;
-                if (e < nt) {
-                    float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
-                    d[0] = v[u].x;
-                    d[1] = v[u].y;
-                    d[2] = v[u].z;
-                    d[3] = v[u].w;
-                }
-            }
+    int s = 0;  // stage index over the launch (barrier parity)
+    // frames f0 .. f0 + F - 1 of the step, or of the list (all CTAs of a cluster agree)
+    auto pass = [&](const int f0, const int F) {
+        if constexpr (kList) {
+            if (tid < F) frame_s[tid] = __ldcg(a.list + f0 + tid);
+            __syncthreads();
         }
-        __syncthreads();
-        const int pf_n = F <= 6 ? 1 : F <= 12 ? 2 : 4, pd_n = F <= 6 ? 1 : 2;
-        const int nob = DO / pd_n, nfb = (F + pf_n - 1) / pf_n;
-        if (tid < nfb * nob) {
-            const int pf = (tid / nob) * pf_n, pd = (tid % nob) * pd_n;
-            if (pf_n == 1) proj_tile<1, 1>(z_s, w_s, pf, pd, F, y_s);
-            else if (pf_n == 2) proj_tile<2, 2>(z_s, w_s, pf, pd, F, y_s);
-            else proj_tile<4, 2>(z_s, w_s, pf, pd, F, y_s);
-        }
-    }
-    __syncthreads();  // the staging is read: the stages take the first slabs
-    if (tid == 0)
-        for (int s = 0; s < NST && s < total; ++s) issue(s);
-    cluster_sync();  // every CTA's projection block is written
+        auto frame_of = [&](int f) {
+            if constexpr (kList) return frame_s[f];
+            else return f0 + f;
+        };
 
-    // r = y, gathered from the cluster's CTAs; the rows past F up to the thread
-    // tile's end are zero (scored, never published)
-    const int rows = (8 / WC) * U;
-    for (int e = tid; e < rows * (kD / 4); e += kThreads) {
-        const int f = e >> 6, d = 4 * (e & 63);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (f < F) v = ld_cluster_f4(cluster_map(smem_u32(y_s + f * YSTRIDE + d % DO), (uint32_t)(d / DO)));
-        *reinterpret_cast<float4*>(r_s + f * RSTRIDE + d) = v;
-    }
-    __syncthreads();
-
-    // this lane's codewords (row within the CTA's slice: cw0 + 8v) and frames (fr0 + u)
-    const int cw0 = wc * 8 * V + g;
-    const int fr0 = wf * U;
-    int s = 0;  // stage index over all levels
-    for (int l = 0; l < a.n_q; ++l) {
-        // minima by level parity: a slot is rewritten two levels later, after the
-        // barrier that every CTA reaches only once it has read it
-        unsigned long long* mk = mk_s + (l & 1) * kClusterMaxBlock;
-        // after the level's scores this lane holds the dots of codewords vq + k, k < V / 4
-        // (see below): their ||c||^2 now, so the loads overlap the scoring
-        const int vq = (w & 1) * (V / 2) + (w >> 1) * (V / 4);
-        float cnv[V / 4];
+        // ---- y = W_in . z for the cluster's F frames x this CTA's DO outputs, each a
+        //      sequential FMA chain over j (the full scan's order); latents and W_in rows
+        //      staged whole (every load in flight at once) over the slab stages and r rows.
+        //      Shared-memory reads bound the chains, so for more than six frames a
+        //      thread keeps 2 or 4 frames x 2 outputs in registers and each value it
+        //      reads feeds several chains; for a few frames, one chain per thread.
+        {
+            const int d0 = rank * DO;
+            constexpr int JS = kDin + 1, J4 = kDin / 4;
+            float* z_s = reinterpret_cast<float*>(sm);   // [F][JS]
+            float* w_s = z_s + F * JS;                   // [DO][JS]
+            const int nz = F * J4, nt = (F + DO) * J4;
+            for (int e0 = tid; e0 < nt; e0 += 16 * kThreads) {
+                float4 v[16];
 #pragma unroll
-        for (int k = 0; k < V / 4; ++k)
-            cnv[k] = __ldg(a.cnorm + (size_t)l * kK + k_base + cw0 + 8 * (vq + k));
-        float acc[U][V];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
-        for (int tt = 0; tt < spl; ++tt, ++s) {
-            mbar_wait(&full[s % NST], (uint32_t)(s / NST) & 1u, abort, a.err);
-#pragma unroll 1
-            for (int jj = 0; jj < nb; ++jj) {
-                // codeword row cw0 + 8v of slab jj: 128 bytes, 16-byte unit x at x ^ (row & 7),
-                // and row & 7 = g
-                const uint8_t* cb = sm + (s % NST) * STAGE_BYTES + jj * slab_bytes + cw0 * 128 + 4 * w;
-                const float* rb = r_s + fr0 * RSTRIDE + (tt * nb + jj) * kSlabDims + w;
-#pragma unroll
-                for (int i = 0; i < kSlabDims; i += 4) {
-                    const int off = ((i >> 2) ^ g) << 4;
-                    float cv[V], rv[U];
-#pragma unroll
-                    for (int v = 0; v < V; ++v) cv[v] = *reinterpret_cast<const float*>(cb + v * 1024 + off);
-#pragma unroll
-                    for (int u = 0; u < U; ++u) rv[u] = rb[u * RSTRIDE + i];
-#pragma unroll
-                    for (int u = 0; u < U; ++u)
-#pragma unroll
-                        for (int v = 0; v < V; ++v) acc[u][v] = fmaf(rv[u], cv[v], acc[u][v]);
-                }
-            }
-            __syncthreads();  // every warp is done with the stage
-            if (tid == 0 && s + NST < total) issue(s + NST);
-        }
-        // dot = (p0 + p1) + (p2 + p3) across the quad as a reduce-scatter: lanes w and
-        // w ^ 1 add their partials of the codeword half each keeps (w & 1 picks it), then
-        // lanes w and w ^ 2 those of the quarter each keeps (w & 2), so lane w ends with
-        // the dots of codewords vq + k, k < V / 4 (3 UV / 4 shuffles instead of 2 UV; the
-        // sums are the same, each addition being commutative). Then the minimum key per
-        // frame over the warp and one slot per warp and frame.
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float h[V / 2];
-#pragma unroll
-            for (int k = 0; k < V / 2; ++k) {
-                const float lo = acc[u][k], hi = acc[u][k + V / 2];
-                const float send = (w & 1) ? lo : hi, keep = (w & 1) ? hi : lo;
-                h[k] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            }
-            unsigned long long best = ~0ull;
-#pragma unroll
-            for (int k = 0; k < V / 4; ++k) {
-                const float a0 = h[k], a1 = h[k + V / 4];
-                const float send = (w & 2) ? a0 : a1, keep = (w & 2) ? a1 : a0;
-                const float dot = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-                best = umin64(best, pack_key(fmaf(-2.f, dot, cnv[k]), k_base + cw0 + 8 * (vq + k)));
-            }
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) best = umin64(best, __shfl_xor_sync(0xffffffffu, best, o));
-            if (lane == 0) red_s[wid * 16 + u] = best;
-        }
-        __syncthreads();
-        // frame f: the minimum over the WC warps that scored its codewords
-        if (tid < F) {
-            const int fw = (tid / U) * WC, fu = tid % U;
-            unsigned long long m = red_s[fw * 16 + fu];
-            for (int c = 1; c < WC; ++c) m = umin64(m, red_s[(fw + c) * 16 + fu]);
-            mk[tid] = m;
-        }
-        cluster_sync();  // every CTA's minima of this level are in its shared memory
-        // winners: the minimum over the cluster's CTAs of each frame
-        if (tid < F) {
-            const uint32_t addr = smem_u32(mk + tid);
-            unsigned long long m[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) m[r] = r < cs ? ld_cluster_u64(cluster_map(addr, (uint32_t)r)) : ~0ull;
-#pragma unroll
-            for (int r = 1; r < 16; ++r) m[0] = umin64(m[0], m[r]);
-            int wn = (int)(uint32_t)m[0];
-            if (wn < 0 || wn >= kK) wn = 0;  // only reachable with NaN / Inf inputs
-            win_s[tid] = wn;
-            if (rank == 0) a.codes[(size_t)(f0 + tid) * a.n_q + l] = (int16_t)wn;
-        }
-        if (l == a.n_q - 1) break;
-        __syncthreads();
-        // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
-        if (l >= 1 || a.variant == 1) {
-            const float* book = a.C32 + (size_t)l * kK * kD;
-            const int ne = F * (kD / 4);
-            for (int e0 = tid; e0 < ne; e0 += 8 * kThreads) {
-                float4 cw[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int e = e0 + u * kThreads;
-                    if (e < ne) cw[u] = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[e >> 6] * kD) + (e & 63));
+                    if (e < nz)
+                        v[u] = load_latent4(a.z, a.dtype, (int64_t)frame_of(e / J4) * kDin + 4 * (e % J4));
+                    else if (e < nt)
+                        v[u] = __ldg(reinterpret_cast<const float4*>(
+                            a.Win32 + (size_t)(d0 + (e - nz) / J4) * kDin + 4 * ((e - nz) % J4)));
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int e = e0 + u * kThreads;
-                    if (e < ne) {
-                        float4* r = reinterpret_cast<float4*>(r_s + (e >> 6) * RSTRIDE + 4 * (e & 63));
-                        float4 v = *r;
-                        v.x -= cw[u].x;
-                        v.y -= cw[u].y;
-                        v.z -= cw[u].z;
-                        v.w -= cw[u].w;
-                        *r = v;
+                    if (e < nt) {
+                        float* d = z_s + (e / J4) * JS + 4 * (e % J4);  // w_s follows z_s
+                        d[0] = v[u].x;
+                        d[1] = v[u].y;
+                        d[2] = v[u].z;
+                        d[3] = v[u].w;
                     }
                 }
             }
+            __syncthreads();
+            const int pf_n = F <= 6 ? 1 : F <= 12 ? 2 : 4, pd_n = F <= 6 ? 1 : 2;
+            const int nob = DO / pd_n, nfb = (F + pf_n - 1) / pf_n;
+            if (tid < nfb * nob) {
+                const int pf = (tid / nob) * pf_n, pd = (tid % nob) * pd_n;
+                if (pf_n == 1) proj_tile<1, 1>(z_s, w_s, pf, pd, F, y_s);
+                else if (pf_n == 2) proj_tile<2, 2>(z_s, w_s, pf, pd, F, y_s);
+                else proj_tile<4, 2>(z_s, w_s, pf, pd, F, y_s);
+            }
         }
-        __syncthreads();  // r updated before the next level's scores
+        __syncthreads();  // the staging is read: the stages take the first slabs
+        if (tid == 0)
+            for (int t = 0; t < NST && t < total; ++t) issue(s + t, t);
+        cluster_sync();  // every CTA's projection block is written
+
+        // r = y, gathered from the cluster's CTAs; the rows past F up to the thread
+        // tile's end are zero (scored, never published)
+        const int rows = (8 / WC) * U;
+        for (int e = tid; e < rows * (kD / 4); e += kThreads) {
+            const int f = e >> 6, d = 4 * (e & 63);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (f < F) v = ld_cluster_f4(cluster_map(smem_u32(y_s + f * YSTRIDE + d % DO), (uint32_t)(d / DO)));
+            *reinterpret_cast<float4*>(r_s + f * RSTRIDE + d) = v;
+        }
+        __syncthreads();
+
+        // this lane's codewords (row within the CTA's slice: cw0 + 8v) and frames (fr0 + u)
+        const int cw0 = wc * 8 * V + g;
+        const int fr0 = wf * U;
+        int tl = 0;  // stage index within the pass
+        for (int l = 0; l < a.n_q; ++l) {
+            // minima by level parity: a slot is rewritten two levels later, after the
+            // barrier that every CTA reaches only once it has read it
+            unsigned long long* mk = mk_s + (l & 1) * kClusterMaxBlock;
+            // after the level's scores this lane holds the dots of codewords vq + k, k < V / 4
+            // (see below): their ||c||^2 now, so the loads overlap the scoring
+            const int vq = (w & 1) * (V / 2) + (w >> 1) * (V / 4);
+            float cnv[V / 4];
+#pragma unroll
+            for (int k = 0; k < V / 4; ++k)
+                cnv[k] = __ldg(a.cnorm + (size_t)l * kK + k_base + cw0 + 8 * (vq + k));
+            float acc[U][V];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[u][v] = 0.f;
+            for (int tt = 0; tt < spl; ++tt, ++s, ++tl) {
+                mbar_wait(&full[s % NST], (uint32_t)(s / NST) & 1u, abort, a.err);
+#pragma unroll 1
+                for (int jj = 0; jj < nb; ++jj) {
+                    // codeword row cw0 + 8v of slab jj: 128 bytes, 16-byte unit x at x ^ (row & 7),
+                    // and row & 7 = g
+                    const uint8_t* cb = sm + (s % NST) * STAGE_BYTES + jj * slab_bytes + cw0 * 128 + 4 * w;
+                    const float* rb = r_s + fr0 * RSTRIDE + (tt * nb + jj) * kSlabDims + w;
+#pragma unroll
+                    for (int i = 0; i < kSlabDims; i += 4) {
+                        const int off = ((i >> 2) ^ g) << 4;
+                        float cv[V], rv[U];
+#pragma unroll
+                        for (int v = 0; v < V; ++v) cv[v] = *reinterpret_cast<const float*>(cb + v * 1024 + off);
+#pragma unroll
+                        for (int u = 0; u < U; ++u) rv[u] = rb[u * RSTRIDE + i];
+#pragma unroll
+                        for (int u = 0; u < U; ++u)
+#pragma unroll
+                            for (int v = 0; v < V; ++v) acc[u][v] = fmaf(rv[u], cv[v], acc[u][v]);
+                    }
+                }
+                __syncthreads();  // every warp is done with the stage
+                if (tid == 0 && tl + NST < total) issue(s + NST, tl + NST);
+            }
+            // dot = (p0 + p1) + (p2 + p3) across the quad as a reduce-scatter: lanes w and
+            // w ^ 1 add their partials of the codeword half each keeps (w & 1 picks it), then
+            // lanes w and w ^ 2 those of the quarter each keeps (w & 2), so lane w ends with
+            // the dots of codewords vq + k, k < V / 4 (3 UV / 4 shuffles instead of 2 UV; the
+            // sums are the same, each addition being commutative). Then the minimum key per
+            // frame over the warp and one slot per warp and frame.
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float h[V / 2];
+#pragma unroll
+                for (int k = 0; k < V / 2; ++k) {
+                    const float lo = acc[u][k], hi = acc[u][k + V / 2];
+                    const float send = (w & 1) ? lo : hi, keep = (w & 1) ? hi : lo;
+                    h[k] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                }
+                unsigned long long best = ~0ull;
+#pragma unroll
+                for (int k = 0; k < V / 4; ++k) {
+                    const float a0 = h[k], a1 = h[k + V / 4];
+                    const float send = (w & 2) ? a0 : a1, keep = (w & 2) ? a1 : a0;
+                    const float dot = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    best = umin64(best, pack_key(fmaf(-2.f, dot, cnv[k]), k_base + cw0 + 8 * (vq + k)));
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) best = umin64(best, __shfl_xor_sync(0xffffffffu, best, o));
+                if (lane == 0) red_s[wid * 16 + u] = best;
+            }
+            __syncthreads();
+            // frame f: the minimum over the WC warps that scored its codewords
+            if (tid < F) {
+                const int fw = (tid / U) * WC, fu = tid % U;
+                unsigned long long m = red_s[fw * 16 + fu];
+                for (int c = 1; c < WC; ++c) m = umin64(m, red_s[(fw + c) * 16 + fu]);
+                mk[tid] = m;
+            }
+            cluster_sync();  // every CTA's minima of this level are in its shared memory
+            // winners: the minimum over the cluster's CTAs of each frame
+            if (tid < F) {
+                const uint32_t addr = smem_u32(mk + tid);
+                unsigned long long m[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) m[r] = r < cs ? ld_cluster_u64(cluster_map(addr, (uint32_t)r)) : ~0ull;
+#pragma unroll
+                for (int r = 1; r < 16; ++r) m[0] = umin64(m[0], m[r]);
+                int wn = (int)(uint32_t)m[0];
+                if (wn < 0 || wn >= kK) wn = 0;  // only reachable with NaN / Inf inputs
+                win_s[tid] = wn;
+                if (rank == 0) a.codes[(size_t)frame_of(tid) * a.n_q + l] = (int16_t)wn;
+            }
+            if (l == a.n_q - 1) break;
+            __syncthreads();
+            // acoustic levels chain on r; variant 1 also starts the chain at y - S_s
+            if (l >= 1 || a.variant == 1) {
+                const float* book = a.C32 + (size_t)l * kK * kD;
+                const int ne = F * (kD / 4);
+                for (int e0 = tid; e0 < ne; e0 += 8 * kThreads) {
+                    float4 cw[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < ne) cw[u] = __ldg(reinterpret_cast<const float4*>(book + (size_t)win_s[e >> 6] * kD) + (e & 63));
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int e = e0 + u * kThreads;
+                        if (e < ne) {
+                            float4* r = reinterpret_cast<float4*>(r_s + (e >> 6) * RSTRIDE + 4 * (e & 63));
+                            float4 v = *r;
+                            v.x -= cw[u].x;
+                            v.y -= cw[u].y;
+                            v.z -= cw[u].z;
+                            v.w -= cw[u].w;
+                            *r = v;
+                        }
+                    }
+                }
+            }
+            __syncthreads();  // r updated before the next level's scores
+        }
+    };
+    if constexpr (kList) {
+        for (int base = 0; base < n_frames; base += nc * a.fc) {
+            const int F = min(a.fc, n_frames - (base + cl * a.fc));
+            if (F > 0) pass(base + cl * a.fc, F);
+        }
+    } else {
+        pass(cl * a.fc, min(a.fc, n_frames - cl * a.fc));  // >= 1 frame: no empty cluster launched
     }
-    if (blockIdx.x == 0 && tid == 0) atomicAdd(&a.stats[0], (unsigned long long)a.B);
+    if (!kList && blockIdx.x == 0 && tid == 0) atomicAdd(&a.stats[0], (unsigned long long)a.B);
     cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
@@ -358,11 +392,13 @@ struct Tile {
 };
 template <int U, int V>
 Tile tile() {
-    return {U, V, reinterpret_cast<const void*>(k_encode_cluster<U, V>)};
+    return {U, V, reinterpret_cast<const void*>(k_encode_cluster<U, V, false>)};
 }
 const Tile kTiles[] = {tile<1, 4>(), tile<2, 4>(), tile<3, 4>(),  tile<4, 4>(),  tile<6, 4>(),
                        tile<8, 4>(), tile<5, 8>(), tile<6, 8>(),  tile<8, 8>(),  tile<9, 8>(),
                        tile<10, 8>(), tile<12, 8>(), tile<14, 8>(), tile<16, 8>()};
+// The list mode's one tile: 32 frames per cluster of 8 (a pass of 32 x clusters frames).
+const void* const kListKernel = reinterpret_cast<const void*>(k_encode_cluster<16, 8, true>);
 
 cudaError_t configure_kernel(const void* k) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -424,6 +460,10 @@ cudaError_t encode_cluster_configure(Tables& t) {
             cudaGetLastError();
             return cudaSuccess;
         }
+    if (configure_kernel(kListKernel) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+    }
     t.cl_max8 = max_clusters(8);
     t.cl_max16 = max_clusters(16);
     return cudaSuccess;
@@ -462,7 +502,8 @@ ClusterPlan plan_encode_cluster(const Tables& t, int B) {
 }
 
 cudaError_t launch_encode_cluster(const Tables& t, const ClusterPlan& p, const void* z, int dtype,
-                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s) {
+                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s,
+                                  bool rescan_list) {
     if (!p.ok) return cudaErrorInvalidValue;
     ClusterArgs a;
     a.C32 = t.C32;
@@ -478,11 +519,15 @@ cudaError_t launch_encode_cluster(const Tables& t, const ClusterPlan& p, const v
     a.cs = p.cs;
     a.fc = p.fc;
     a.codes = codes;
+    a.list = rescan_list ? t.rescan_list : nullptr;
+    a.list_count = rescan_list ? t.rescan_count : nullptr;
+    a.list_cap = (int)kRescanCapacity;
     cudaLaunchAttribute at[1];
     const cudaLaunchConfig_t cfg = launch_config(p.nc * p.cs, p.cs, s, at);
     const CUtensorMap* tm = p.cs == 8 ? &t.tm_C32_8 : &t.tm_C32_16;
     void* args[] = {const_cast<CUtensorMap*>(tm), &a};
-    return cudaLaunchKernelExC(&cfg, kTiles[p.tile].kernel, args);
+    if (rescan_list && !(p.cs == 8 && p.U == 16 && p.V == 8)) return cudaErrorInvalidConfiguration;
+    return cudaLaunchKernelExC(&cfg, rescan_list ? kListKernel : kTiles[p.tile].kernel, args);
 }
 
 }  // namespace mimi

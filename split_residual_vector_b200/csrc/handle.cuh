@@ -139,9 +139,12 @@ struct ClusterPlan {
 // for a cluster size the device cannot run; not an error)
 cudaError_t encode_cluster_configure(Tables& t);
 ClusterPlan plan_encode_cluster(const Tables& t, int B);
-// Reads only the tables: launches on several streams may overlap.
+// Frames 0..B-1 read only the tables: launches on several streams may overlap.
+// rescan_list: encode the frames of t.rescan_list (count on the device) instead, nc x fc
+// per pass of the launch (plan for B = kClusterMaxBlock x clusters; B itself unused).
 cudaError_t launch_encode_cluster(const Tables& t, const ClusterPlan& p, const void* z, int dtype,
-                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s);
+                                  int B, int n_q, int variant, int16_t* codes, cudaStream_t s,
+                                  bool rescan_list = false);
 // selftest.cu: a kernel whose wait can never complete (which 0: an mbarrier,
 // as the tensor-core encoder waits; 1: a group barrier, as the wide encoder
 // waits); it times out after ~50 ms and records MIMI_DEV_ERR_TIMEOUT.
