@@ -208,6 +208,19 @@ int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st *stream);
 int mimi_rvq_wait_selftest(mimi_rvq_t h, int which, struct CUstream_st *stream);
 
 /*
+ * Turn the thread-block-cluster form of the float32 latency encoder on (enabled = 1,
+ * the default where the device runs clusters) or off (0). Off, streaming steps of
+ * up to 256 frames and the float32 re-encode after a batch encode run the group form
+ * instead (CTAs of a cooperative launch meeting at barriers in global memory: slower,
+ * same codes), as on a device without clusters. Host-side setting of the handle, read
+ * by the calls issued after it; not to be changed while another thread issues calls
+ * on the handle. Returns MIMI_RVQ_OK, or MIMI_RVQ_EINVAL for a NULL handle or an
+ * enabled value other than 0 or 1. Turning it on where the device runs no clusters
+ * changes nothing.
+ */
+int mimi_rvq_set_cluster_form(mimi_rvq_t h, int enabled);
+
+/*
  * Counters since create (synchronises `stream`): frames encoded, and frames
  * whose bf16 candidate pass could not certify its candidate set at some level
  * and were resolved in float32 instead (re-encoded by the full scan after a

@@ -76,6 +76,8 @@ def library() -> ctypes.CDLL:
     lib.mimi_rvq_encode_step_ex.restype = ci
     lib.mimi_rvq_wait_selftest.argtypes = [vp, ci, vp]
     lib.mimi_rvq_wait_selftest.restype = ci
+    lib.mimi_rvq_set_cluster_form.argtypes = [vp, ci]
+    lib.mimi_rvq_set_cluster_form.restype = ci
     i32 = ctypes.c_int32
     lib.mimi_rvq_delay_pack.argtypes = [vp, vp, ci, i64, vp, i64, i32, i32, vp, vp]
     lib.mimi_rvq_delay_pack.restype = ci
@@ -245,6 +247,13 @@ class Quantizer:
         times out after ~50 ms. The next get_error() returns -6 (timed out)."""
         _check(library().mimi_rvq_wait_selftest(self._h, int(which), _stream(stream)),
                "mimi_rvq_wait_selftest")
+
+    def set_cluster_form(self, enabled: bool):
+        """Use the thread-block-cluster form of the float32 latency encoder (default where the
+        device runs clusters) or the group form, for streaming steps of up to 256 frames and
+        the float32 re-encode after a batch encode."""
+        _check(library().mimi_rvq_set_cluster_form(self._h, 1 if enabled else 0),
+               "mimi_rvq_set_cluster_form")
 
     def get_error(self, stream=None) -> int:
         """Synchronise the stream; return and clear the device error status (0 = ok)."""

@@ -19,6 +19,7 @@ struct mimi_rvq {
     int device = 0;
     int num_sms = 148;
     mimi::Tables t;
+    int cl_max8 = 0, cl_max16 = 0;  // the device's cluster counts (t's are 0 while the form is off)
 };
 
 namespace {
@@ -229,6 +230,8 @@ int mimi_rvq_create(const float* codebooks, const float* W_in, const float* W_ou
     // the cluster form needs its slab maps; a size without one stays off
     if (!make_tmap_slabs(&t.tm_C32_8, t.C32, (uint64_t)kQ * kK, kK / 8)) t.cl_max8 = 0;
     if (!make_tmap_slabs(&t.tm_C32_16, t.C32, (uint64_t)kQ * kK, kK / 16)) t.cl_max16 = 0;
+    h->cl_max8 = t.cl_max8;
+    h->cl_max16 = t.cl_max16;
     *out = h;
     return MIMI_RVQ_OK;
 }
@@ -355,6 +358,13 @@ int mimi_rvq_wait_selftest(mimi_rvq_t h, int which, struct CUstream_st* stream) 
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MIMI_RVQ_EINVAL;
     return from_cuda(mimi::launch_wait_selftest(h->t, which, stream));
+}
+
+int mimi_rvq_set_cluster_form(mimi_rvq_t h, int enabled) {
+    if (!h || (enabled != 0 && enabled != 1)) return MIMI_RVQ_EINVAL;
+    h->t.cl_max8 = enabled ? h->cl_max8 : 0;
+    h->t.cl_max16 = enabled ? h->cl_max16 : 0;
+    return MIMI_RVQ_OK;
 }
 
 int mimi_rvq_get_error(mimi_rvq_t h, struct CUstream_st* stream) {

@@ -185,6 +185,55 @@ def test_small_streaming_steps_equal_the_full_scan(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_group_form_steps_equal_the_full_scan(dtype):
+    """With the cluster form off (as on a device without clusters) steps of at most 256
+    frames run the group form of the latency encoder (groups of up to 64 frames over CTAs
+    meeting at barriers in global memory): its codes equal encode_scan's too, for one to four
+    groups, ragged tails and every thread tile, also under CUDA-graph replay."""
+    model, frames = synth.streaming_step(256, calls=2)
+    q = quantizer(model)
+    q.set_cluster_form(False)
+    z = frames[0] if dtype == "f32" else synth.to_bf16_bits(frames[0])
+    zd = to_device(np.ascontiguousarray(z))
+    sizes = (1, 2, 15, 16, 17, 33, 63, 64, 65, 127, 128, 129, 200, 255, 256)
+    for b in sizes:
+        step = q.encode_step(zd[:b]).cpu().numpy()
+        scan = q.encode_scan(zd[:b]).cpu().numpy()
+        assert np.array_equal(step, scan), f"B={b}: {np.argwhere(step != scan)[:5]}"
+    out = torch.empty((128, 8), dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        q.encode_step(zd[:128], out=out, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    static_in = zd[:128].clone()
+    with torch.cuda.graph(g):
+        q.encode_step(static_in, out=out, stream=torch.cuda.current_stream())
+    for call in range(2):
+        zc = frames[call][:128] if dtype == "f32" else synth.to_bf16_bits(frames[call][:128])
+        static_in.copy_(to_device(np.ascontiguousarray(zc)))
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(out.cpu().numpy(), q.encode_scan(static_in).cpu().numpy())
+    q.set_cluster_form(True)
+    assert np.array_equal(q.encode_step(zd[:100]).cpu().numpy(), q.encode_scan(zd[:100]).cpu().numpy())
+    assert q.get_error() == 0
+
+
+def test_cluster_form_switch_rejects_bad_values():
+    model, _ = synth.streaming_step(1, calls=1)
+    q = quantizer(model)
+    import split_residual_vector_b200 as pkg
+    lib = pkg.library()
+    assert lib.mimi_rvq_set_cluster_form(None, 1) == -1
+    assert lib.mimi_rvq_set_cluster_form(q._h, 2) == -1
+    assert lib.mimi_rvq_set_cluster_form(q._h, 0) == 0
+    assert lib.mimi_rvq_set_cluster_form(q._h, 1) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_sliced_streaming_steps_match_the_oracle(dtype):
     """Steps of more than 480 frames run the codebook-sliced tensor-core encoder (8 CTAs per
     128-frame group, candidate lists exchanged through global memory): codes equal the
@@ -395,14 +444,17 @@ def test_self_profile_counts(offline_small):
     assert prof["cta_total"] > 0 and prof["epi_scan"] > 0
 
 
-def test_rescan_of_many_frames_in_several_batches():
+@pytest.mark.parametrize("cluster_form", [True, False])
+def test_rescan_of_many_frames_in_several_batches(cluster_form):
     """Every level-1 codeword has ~20 exact copies, so no frame's candidate window can be
-    certified and all 2500 frames are re-encoded by the float32 wide encoder, 1024 at a time
-    (three batches). Its scores are the full scan's, so the codes equal encode_scan's; they
-    also match the oracle (ties between copies go to the lowest index on both sides)."""
+    certified and all 2500 frames are re-encoded by the float32 latency encoder: the cluster
+    form in passes of 32 frames per cluster, or the group form 1024 at a time (three
+    batches). Its scores are the full scan's, so the codes equal encode_scan's; they also
+    match the oracle (ties between copies go to the lowest index on both sides)."""
     model = _small_model(seed=33)
     model.C[1] = model.C[1][np.arange(2048) % 100]
     q = quantizer(model)
+    q.set_cluster_form(cluster_form)
     rng = np.random.default_rng(34)
     z = rng.standard_normal((2500, 512)).astype(np.float32)
     zd = to_device(z)
