@@ -378,6 +378,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         pass(cl * a.fc, min(a.fc, n_frames - cl * a.fc));  // >= 1 frame: no empty cluster launched
     }
+    // a wait that ran out (the error flag is set) may have left its stage's copy in flight:
+    // wait for the last stages' copies (bounded) so that none lands after the CTA exits
+    if (*abort && tid == 0) {
+        for (int k = s > NST ? s - NST : 0; k < s; ++k) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full[k % NST], (uint32_t)(k / NST) & 1u) &&
+                   clock64() - t0 < kWaitBudgetCycles) {
+            }
+        }
+    }
     if (!kList && blockIdx.x == 0 && tid == 0) atomicAdd(&a.stats[0], (unsigned long long)a.B);
     cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
