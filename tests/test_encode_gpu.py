@@ -464,6 +464,11 @@ def test_rescan_of_many_frames_in_several_batches(cluster_form):
     assert np.array_equal(codes, q.encode_scan(zd).cpu().numpy())
     ref, db, ds = oracle.encode(z, model.W_in, model.C)
     assert_codes_match(codes, ref, db, ds, "all frames re-scanned")
+    # the re-encode with fewer codebooks and with the acoustic chain on y - S_s
+    for n_q, variant in ((3, 0), (5, 1)):
+        got = q.encode(zd[:700], n_q=n_q, variant=variant).cpu().numpy()
+        want = q.encode_scan(zd[:700], n_q=n_q, variant=variant).cpu().numpy()
+        assert np.array_equal(got, want), f"n_q={n_q} variant={variant}"
     assert q.get_error() == 0
 
 
